@@ -1,0 +1,403 @@
+"""Pins for the fp64 oracle: each test ties it to something other than itself.
+
+Brute-force enumeration, closed forms, hand calculations with the ``math`` module, reduction to a
+dense matrix product, central finite differences, symmetry (translation, rotation, permutation),
+replica additivity and the exact zero at the cutoff. A plausible mistake in the oracle (a dropped
+bias, a wrong sign, a transposed weight, a missed neighbor) fails at least one of them.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import schnet
+from atomistic_neighbor_list_b200 import synth
+
+
+def small_model(F=8, R=6, n_blocks=2, r_c=5.0, seed=7, n_heads=2, head_dim=4, n_types=3):
+    wl = synth.Workload("t", "energy_forces", 0, r_c, R, F, "fp32", n_blocks=n_blocks,
+                        n_types=n_types, n_heads=n_heads, head_dim=head_dim)
+    w = synth.make_weights(wl, seed=seed)
+    return oracle.Model.from_workload(wl, w), w, wl
+
+
+# ----------------------------------------------------------------------------- neighbor list
+def brute_csr(pos, r_c, graph_ptr=None):
+    """O(N^2) enumeration with plain Python floats (IEEE double, same operation order)."""
+    pos = np.asarray(pos, dtype=np.float32)
+    n = len(pos)
+    gp = [0, n] if graph_ptr is None else list(graph_ptr)
+    graph_of = np.zeros(n, dtype=np.int64)
+    for g in range(len(gp) - 1):
+        graph_of[gp[g]:gp[g + 1]] = g
+    rc = float(np.float32(r_c))
+    rc2 = rc * rc
+    P = [tuple(float(c) for c in p) for p in pos]
+    row_ptr, cols = [0], []
+    for i in range(n):
+        xi, yi, zi = P[i]
+        for j in range(n):
+            if j == i or graph_of[j] != graph_of[i]:
+                continue
+            xj, yj, zj = P[j]
+            dx, dy, dz = xj - xi, yj - yi, zj - zi
+            if (dx * dx + dy * dy) + dz * dz < rc2:
+                cols.append(j)
+        row_ptr.append(len(cols))
+    return np.array(row_ptr, dtype=np.int32), np.array(cols, dtype=np.int32)
+
+
+@pytest.mark.parametrize("n", [1, 2, 33, 300])
+def test_csr_matches_brute_force_uniform(n):
+    pos = synth.uniform_positions(n, seed=n)
+    rp, ci = oracle.neighbor_csr(pos, 5.0)
+    brp, bci = brute_csr(pos, 5.0)
+    assert np.array_equal(rp, brp) and np.array_equal(ci, bci)
+
+
+def test_csr_matches_brute_force_chains():
+    pos, gp = synth.chain_replicas(3, 120, seed=5)
+    rp, ci = oracle.neighbor_csr(pos, 10.0, gp)
+    brp, bci = brute_csr(pos, 10.0, gp)
+    assert np.array_equal(rp, brp) and np.array_equal(ci, bci)
+    # no edge leaves its replica
+    dst = np.repeat(np.arange(len(pos)), np.diff(rp))
+    assert np.array_equal(dst // 120, ci // 120)
+
+
+def test_csr_matches_brute_force_vectorised_1500():
+    pos = synth.uniform_positions(1500, seed=11)
+    rp, ci = oracle.neighbor_csr(pos, 5.0)
+    p = pos.astype(np.float64)
+    cols, row_ptr = [], [0]
+    for i in range(len(p)):
+        dx, dy, dz = p[:, 0] - p[i, 0], p[:, 1] - p[i, 1], p[:, 2] - p[i, 2]
+        d2 = (dx * dx + dy * dy) + dz * dz
+        js = np.nonzero(d2 < 25.0)[0]
+        js = js[js != i]
+        cols.extend(js.tolist())
+        row_ptr.append(len(cols))
+    assert np.array_equal(rp, np.array(row_ptr)) and np.array_equal(ci, np.array(cols))
+
+
+def test_csr_sorted_symmetric_no_self():
+    pos = synth.uniform_positions(2000, seed=3)
+    rp, ci = oracle.neighbor_csr(pos, 5.0)
+    n = len(pos)
+    dst = np.repeat(np.arange(n), np.diff(rp))
+    assert np.all(ci != dst)
+    for i in range(n):
+        row = ci[rp[i]:rp[i + 1]]
+        assert np.all(np.diff(row) > 0)
+    fwd = set(zip(dst.tolist(), ci.tolist()))
+    assert all((j, i) in fwd for (i, j) in fwd)
+
+
+def test_interior_degree_matches_density():
+    # interior atoms of a uniform cube see rho * 4/3 pi r_c^3 = 52.36 neighbors on average
+    pos = synth.uniform_positions(10_000, seed=0)
+    rp, _ = oracle.neighbor_csr(pos, 5.0)
+    L = synth.box_length(10_000)
+    inner = np.all((pos > 5.0) & (pos < L - 5.0), axis=1)
+    mean = np.diff(rp)[inner].mean()
+    import json, os
+    facts = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "workload_facts.json")))
+    want = facts["interior_mean_degree_uniform_0.1_per_A3_rc5"]["value"]
+    assert abs(want - 0.1 * 4.0 / 3.0 * math.pi * 125.0) < 1e-9
+    assert abs(mean - want) < 1.5
+
+
+def test_pair_exactly_at_cutoff_excluded():
+    pos = np.array([[0, 0, 0], [5, 0, 0]], dtype=np.float32)
+    rp, ci = oracle.neighbor_csr(pos, 5.0)
+    assert rp.tolist() == [0, 0, 0] and len(ci) == 0
+    pos[1, 0] = np.float32(4.9999)
+    rp, ci = oracle.neighbor_csr(pos, 5.0)
+    assert rp.tolist() == [0, 1, 2] and ci.tolist() == [1, 0]
+
+
+def test_padded_list_keeps_nearest_k():
+    pos = synth.uniform_positions(600, seed=4)
+    K = 20
+    nbr, mask = oracle.neighbor_padded(pos, 5.0, K)
+    rp, ci = brute_csr(pos, 5.0)
+    p = pos.astype(np.float64)
+    for i in range(len(pos)):
+        full = ci[rp[i]:rp[i + 1]]
+        if len(full) <= K:
+            want = full
+        else:
+            key = sorted(((float(((p[j, 0] - p[i, 0]) ** 2 + (p[j, 1] - p[i, 1]) ** 2)
+                                 + (p[j, 2] - p[i, 2]) ** 2), int(j)) for j in full))
+            want = np.sort(np.array([j for _, j in key[:K]]))
+        cnt = int(mask[i].sum())
+        assert cnt == len(want)
+        assert np.array_equal(nbr[i, :cnt], want)
+        assert np.all(nbr[i, cnt:] == -1) and np.all(mask[i, cnt:] == 0)
+
+
+# ----------------------------------------------------------------------------- element functions
+def test_rbf_closed_forms():
+    mu = oracle.rbf_centres(50, 0.0, 5.0)
+    assert mu[0] == 0.0 and abs(mu[-1] - 5.0) < 1e-15 and abs(mu[1] - 5.0 / 49) < 1e-15
+    e = oracle.gaussian_rbf(mu, mu, 10.0)
+    assert np.allclose(np.diag(e), 1.0, rtol=0, atol=0)
+    d = np.array([1.234])
+    assert abs(oracle.gaussian_rbf(d, mu, 10.0)[0, 7] - math.exp(-10.0 * (1.234 - mu[7]) ** 2)) < 1e-15
+    h = 1e-6
+    fd = (oracle.gaussian_rbf(d + h, mu, 10.0) - oracle.gaussian_rbf(d - h, mu, 10.0)) / (2 * h)
+    assert np.allclose(oracle.gaussian_rbf_grad(d, mu, 10.0), fd, atol=1e-8)
+
+
+def test_cosine_cutoff_closed_forms():
+    rc = 5.0
+    f = oracle.cosine_cutoff(np.array([0.0, 2.5, 5.0, 5.5, 100.0]), rc)
+    assert f[0] == 1.0 and abs(f[1] - 0.5) < 1e-15
+    assert f[2] == 0.0 and f[3] == 0.0 and f[4] == 0.0  # exactly zero at and beyond the cutoff
+    g = oracle.cosine_cutoff_grad(np.array([0.0, 2.5, 5.0, 6.0]), rc)
+    assert g[0] == 0.0 and abs(g[1] + math.pi / (2 * rc)) < 1e-15 and g[2] == 0.0 and g[3] == 0.0
+    d = np.array([1.1, 3.3, 4.9])
+    h = 1e-6
+    fd = (oracle.cosine_cutoff(d + h, rc) - oracle.cosine_cutoff(d - h, rc)) / (2 * h)
+    assert np.allclose(oracle.cosine_cutoff_grad(d, rc), fd, atol=1e-9)
+
+
+def test_ssp_closed_forms():
+    assert oracle.ssp(0.0) == 0.0
+    assert abs(oracle.ssp_grad(0.0) - 0.5) < 1e-16
+    for x in [-30.0, -3.0, -0.7, 0.2, 1.5, 4.0, 20.0]:
+        assert abs(oracle.ssp(x) - math.log(0.5 * math.exp(x) + 0.5)) < 1e-14 * max(1, abs(x))
+    assert abs(oracle.ssp(60.0) - (60.0 - math.log(2.0))) < 1e-12
+    assert abs(oracle.ssp(-60.0) + math.log(2.0)) < 1e-12
+    x = np.linspace(-6, 6, 25)
+    fd = (oracle.ssp(x + 1e-6) - oracle.ssp(x - 1e-6)) / 2e-6
+    assert np.allclose(oracle.ssp_grad(x), fd, atol=1e-8)
+
+
+# ----------------------------------------------------------------------------- filter and cfconv
+def test_filter_with_zero_first_layer_by_hand():
+    model, w, wl = small_model()
+    model.w["A1.0"][:] = 0.0
+    d = 3.1
+    c1, A2, c2 = w["c1.0"].astype(float), w["A2.0"].astype(float), w["c2.0"].astype(float)
+    fc = 0.5 * (math.cos(math.pi * d / 5.0) + 1.0)
+    F = wl.F
+    want = []
+    for f in range(F):
+        acc = float(c2[f])
+        for g in range(F):
+            acc += math.log(0.5 * math.exp(float(c1[g])) + 0.5) * float(A2[g, f])
+        want.append(fc * acc)
+    got = oracle.filter_weights(model, 0, np.array([d]))[0]
+    assert np.allclose(got, want, rtol=1e-13, atol=1e-14)
+
+
+def test_two_atom_cfconv_by_hand():
+    model, w, wl = small_model(F=4, R=5)
+    pos = np.array([[0.1, 0.2, 0.3], [1.0, 2.0, 2.5]], dtype=np.float32)
+    x = synth.node_features(2, 4, seed=9)
+    rp, ci = oracle.neighbor_csr(pos, 5.0)
+    m = oracle.cfconv(model, 0, pos, rp, ci, x)
+    p = pos.astype(float)
+    d = math.sqrt(sum((p[0, c] - p[1, c]) ** 2 for c in range(3)))
+    mu = [5.0 * k / 4 for k in range(5)]
+    e = [math.exp(-10.0 * (d - mu[k]) ** 2) for k in range(5)]
+    A1, c1, A2, c2 = (w[k].astype(float) for k in ("A1.0", "c1.0", "A2.0", "c2.0"))
+    h1 = [math.log(0.5 * math.exp(sum(e[k] * A1[k, g] for k in range(5)) + c1[g]) + 0.5)
+          for g in range(4)]
+    fc = 0.5 * (math.cos(math.pi * d / 5.0) + 1.0)
+    W = [fc * (sum(h1[g] * A2[g, f] for g in range(4)) + c2[f]) for f in range(4)]
+    assert np.allclose(m[0], [x[1, f] * W[f] for f in range(4)], rtol=1e-12, atol=1e-14)
+    assert np.allclose(m[1], [x[0, f] * W[f] for f in range(4)], rtol=1e-12, atol=1e-14)
+
+
+def test_cfconv_reduces_to_dense_spmm():
+    # A1 = A2 = 0, c2 = 1  =>  W_ij = f_c(d_ij)  =>  m = A x with A_ij = f_c(d_ij) on neighbor pairs
+    model, w, wl = small_model(F=8)
+    model.w["A1.0"][:] = 0
+    model.w["A2.0"][:] = 0
+    model.w["c2.0"][:] = 1
+    pos = synth.uniform_positions(150, seed=2)
+    x = synth.node_features(150, 8, seed=1)
+    rp, ci = brute_csr(pos, 5.0)
+    A = np.zeros((150, 150))
+    p = pos.astype(float)
+    for i in range(150):
+        for j in ci[rp[i]:rp[i + 1]]:
+            d = math.sqrt(sum((p[i, c] - p[j, c]) ** 2 for c in range(3)))
+            A[i, j] = 0.5 * (math.cos(math.pi * d / 5.0) + 1.0)
+    m = oracle.cfconv(model, 0, pos, rp, ci, x)
+    assert np.allclose(m, A @ x.astype(float), rtol=1e-12, atol=1e-12)
+
+
+def test_cfconv_empty_rows_and_permutation():
+    model, w, wl = small_model(F=8)
+    pos = synth.uniform_positions(120, seed=5)
+    pos[7] = [500.0, 500.0, 500.0]  # isolated atom -> empty row
+    x = synth.node_features(120, 8, seed=2)
+    rp, ci = oracle.neighbor_csr(pos, 5.0)
+    m = oracle.cfconv(model, 0, pos, rp, ci, x)
+    assert rp[8] == rp[7] and np.all(m[7] == 0.0)
+    perm = np.random.default_rng(0).permutation(120)
+    rp2, ci2 = oracle.neighbor_csr(pos[perm], 5.0)
+    m2 = oracle.cfconv(model, 0, pos[perm], rp2, ci2, x[perm])
+    assert np.allclose(m2, m[perm], rtol=1e-12, atol=1e-12)
+    # sampled rows equal the same rows of the full computation
+    rows = np.array([3, 7, 50, 119])
+    assert np.array_equal(oracle.cfconv(model, 0, pos, rp, ci, x, rows=rows), m[rows])
+
+
+# ----------------------------------------------------------------------------- energy and forces
+@pytest.fixture(scope="module")
+def fd_system():
+    wl = synth.WORKLOADS["fd64"]
+    w = synth.make_weights(wl)
+    model = oracle.Model.from_workload(wl, w)
+    pos = synth.uniform_positions(64, seed=0)
+    types = synth.atom_types(64, wl.n_types)
+    rp, ci = oracle.neighbor_csr(pos, wl.r_c)
+    return model, pos, types, rp, ci
+
+
+def test_forces_match_central_differences(fd_system):
+    model, pos, types, rp, ci = fd_system
+    E, F = oracle.energy_forces(model, pos, types, rp, ci)
+    p0 = pos.astype(np.float64)
+    h = 1e-3
+    fd = np.zeros_like(p0)
+    for a in range(len(p0)):
+        for c in range(3):
+            pp, pm = p0.copy(), p0.copy()
+            pp[a, c] += h
+            pm[a, c] -= h
+            ep = oracle.energies(model, pp, types, rp, ci)[0]
+            em = oracle.energies(model, pm, types, rp, ci)[0]
+            fd[a, c] = -(ep - em) / (2 * h)
+    rel = np.linalg.norm(fd - F) / np.linalg.norm(F)
+    assert rel < 1e-5, rel
+
+
+def test_force_forms_agree_and_momentum_zero(fd_system):
+    model, pos, types, rp, ci = fd_system
+    E1, F1 = oracle.energy_forces(model, pos, types, rp, ci, method="scatter")
+    E2, F2 = oracle.energy_forces(model, pos, types, rp, ci, method="pair")
+    assert np.array_equal(E1, E2)
+    scale = np.abs(F1).max()
+    assert np.max(np.abs(F1 - F2)) <= 1e-12 * scale
+    assert np.max(np.abs(F1.sum(axis=0))) <= 1e-12 * scale * len(pos)
+    torque = np.cross(pos.astype(float), F1).sum(axis=0)
+    assert np.max(np.abs(torque)) <= 1e-11 * scale * len(pos) * 10
+
+
+def test_rotation_translation_invariance(fd_system):
+    model, pos, types, rp, ci = fd_system
+    E, F = oracle.energy_forces(model, pos, types, rp, ci)
+    rng = np.random.default_rng(42)
+    Q, _ = np.linalg.qr(rng.normal(size=(3, 3)))
+    if np.linalg.det(Q) < 0:
+        Q[:, 0] = -Q[:, 0]
+    assert abs(np.linalg.det(Q) - 1.0) < 1e-12
+    t = rng.normal(size=3) * 10
+    p2 = pos.astype(np.float64) @ Q.T + t
+    rp2, ci2 = oracle.neighbor_csr(p2, 5.0)
+    E2, F2 = oracle.energy_forces(model, p2, types, rp2, ci2)
+    assert abs(E2[0] - E[0]) <= 1e-10 * abs(E[0])
+    assert np.max(np.abs(F2 - F @ Q.T)) <= 1e-9 * np.abs(F).max()
+
+
+def test_replica_additivity_and_isolation():
+    model, w, wl = small_model(F=8, R=6, n_blocks=2, r_c=10.0)
+    pos, gp = synth.chain_replicas(3, 60, seed=1)
+    types = synth.atom_types(len(pos), wl.n_types)
+    rp, ci = oracle.neighbor_csr(pos, 10.0, gp)
+    E, F = oracle.energy_forces(model, pos, types, rp, ci, gp)
+    for g in range(3):
+        sl = slice(gp[g], gp[g + 1])
+        rpg, cig = oracle.neighbor_csr(pos[sl], 10.0)
+        Eg, Fg = oracle.energy_forces(model, pos[sl], types[sl], rpg, cig)
+        assert abs(Eg[0] - E[g]) <= 1e-12 * max(1.0, abs(E[g]))
+        assert np.allclose(Fg, F[sl], rtol=1e-11, atol=1e-12)
+
+
+def test_exact_zero_at_cutoff():
+    model, w, wl = small_model(F=8)
+    types = np.array([0, 1], dtype=np.int32)
+    pos = np.array([[0, 0, 0], [5, 0, 0]], dtype=np.float32)
+    rp, ci = oracle.neighbor_csr(pos, 5.0)
+    E, F = oracle.energy_forces(model, pos, types, rp, ci)
+    assert np.all(F == 0.0)
+    x = synth.node_features(2, 8)
+    assert np.all(oracle.cfconv(model, 0, pos, rp, ci, x) == 0.0)
+    # the same pair pushed just inside: small but non-zero force along x only
+    pos[1, 0] = np.float32(5.0 - 1e-3)
+    rp, ci = oracle.neighbor_csr(pos, 5.0)
+    E2, F2 = oracle.energy_forces(model, pos, types, rp, ci)
+    assert 0 < np.abs(F2[:, 0]).max() < 1e-3 and np.all(F2[:, 1:] == 0.0)
+    assert abs(E2[0] - E[0]) < 1e-4
+
+
+# ----------------------------------------------------------------------------- attention
+def test_attention_uniform_weights_give_mean():
+    model, w, wl = small_model(F=8, n_heads=2, head_dim=4)
+    for k in ("Wq", "Wk", "P", "p"):
+        model.w[k][:] = 0
+    pos = synth.uniform_positions(80, seed=8)
+    x = synth.node_features(80, 8, seed=4)
+    nbr, mask = oracle.neighbor_padded(pos, 5.0, 16)
+    out = oracle.attention(model, pos, nbr, mask, x)
+    rp, ci = brute_csr(pos, 5.0)
+    for i in range(80):
+        cnt = int(mask[i].sum())
+        if cnt == 0:
+            assert np.all(out[i] == 0)
+            continue
+        js = nbr[i, :cnt]
+        W = oracle.filter_weights(model, 0, np.linalg.norm(pos[i].astype(float) - pos[js], axis=1))
+        assert np.allclose(out[i], (x[js] * W).mean(axis=0), rtol=1e-12, atol=1e-13)
+
+
+def test_attention_two_neighbors_by_hand():
+    model, w, wl = small_model(F=4, R=5, n_heads=2, head_dim=2)
+    pos = np.array([[0, 0, 0], [1.5, 0.5, 0], [0, 2.5, 1.0], [40, 40, 40]], dtype=np.float32)
+    x = synth.node_features(4, 4, seed=6)
+    nbr = np.array([[1, 2, -1], [0, -1, -1], [0, -1, -1], [-1, -1, -1]], dtype=np.int32)
+    mask = (nbr >= 0).astype(np.uint8)
+    out = oracle.attention(model, pos, nbr, mask, x)
+    W64 = {k: v.astype(float) for k, v in w.items()}
+    p = pos.astype(float)
+    xf = x.astype(float)
+    q = [[sum(xf[0, a] * W64["Wq"][a, f] for a in range(4)) for f in range(4)]]
+    kk = [[sum(xf[j, a] * W64["Wk"][a, f] for a in range(4)) for f in range(4)] for j in range(4)]
+    mu = [5.0 * k / 4 for k in range(5)]
+    logits, vals = [], []
+    for j in (1, 2):
+        d = math.sqrt(sum((p[0, c] - p[j, c]) ** 2 for c in range(3)))
+        e = [math.exp(-10.0 * (d - mu[k]) ** 2) for k in range(5)]
+        Wf = oracle.filter_weights(model, 0, np.array([d]))[0]
+        vals.append([xf[j, f] * Wf[f] for f in range(4)])
+        logits.append([sum(q[0][h * 2 + c] * kk[j][h * 2 + c] for c in range(2)) / math.sqrt(2)
+                       + sum(e[k] * W64["P"][k, h] for k in range(5)) + W64["p"][h]
+                       for h in range(2)])
+    want = []
+    for h in range(2):
+        a = [math.exp(logits[0][h]), math.exp(logits[1][h])]
+        s = a[0] + a[1]
+        for c in range(2):
+            f = h * 2 + c
+            want.append((a[0] * vals[0][f] + a[1] * vals[1][f]) / s)
+    assert np.allclose(out[0], want, rtol=1e-12, atol=1e-14)
+    W1 = oracle.filter_weights(model, 0, np.array([np.linalg.norm(p[1] - p[0])]))[0]
+    assert np.allclose(out[1], xf[0] * W1, rtol=1e-12)  # one valid neighbor: alpha = 1
+    assert np.all(out[3] == 0.0)  # no valid neighbor: zero row
+
+
+def test_attention_logit_shift_invariance():
+    model, w, wl = small_model(F=8, n_heads=2, head_dim=4)
+    pos = synth.uniform_positions(60, seed=3)
+    x = synth.node_features(60, 8, seed=2)
+    nbr, mask = oracle.neighbor_padded(pos, 5.0, 12)
+    o1 = oracle.attention(model, pos, nbr, mask, x)
+    model.w["p"] = model.w["p"] + 3.0
+    o2 = oracle.attention(model, pos, nbr, mask, x)
+    assert np.allclose(o1, o2, rtol=1e-12, atol=1e-13)
