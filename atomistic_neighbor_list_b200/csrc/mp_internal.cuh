@@ -1,0 +1,170 @@
+// Internal declarations of libmp: context layout, kernel launch/profiling helper, device helpers.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <vector>
+
+#include "../../include/mp.h"
+
+namespace mp {
+
+constexpr int kMaxR = 64;   // radial functions supported by the kernels
+
+// Device-status bits raised by kernels (read and cleared by mp_status_sync).
+enum : int { kStatusBounds = 1, kStatusCapacity = 2, kStatusTimeout = 4 };
+
+// Radial-basis and envelope parameters of the model.
+struct Radial {
+  int R;
+  float gamma, mu_min, dmu, r_c;
+};
+
+// Filter-MLP weights of one block (device, fp32 values; bf16-rounded under MP_BF16).
+struct FilterW {
+  const float* A1;  // [R][F]
+  const float* c1;  // [F]
+  const float* A2;  // [F][F]
+  const float* c2;  // [F]
+};
+
+// Kernel identities for launch counting and per-kernel timing.
+enum KernelId : int {
+  K_EMBED = 0, K_DENSE, K_READOUT_E, K_READOUT_BWD, K_GRAPH_SUM, K_CFCONV_FWD_SIMT,
+  K_CFCONV_BWD_SIMT, K_ATTN_SIMT, K_VALIDATE, K_CFCONV_FWD_TC, K_CFCONV_BWD_TC, K_ATTN_TC,
+  K_NUM
+};
+const char* kernel_name(int id);
+
+}  // namespace mp
+
+struct mp_ctx {
+  mp_config cfg;
+  int device = 0;
+  int num_sms = 148;
+  // weights (device, fp32; values bf16-rounded under MP_BF16)
+  float* emb = nullptr;
+  float *A1[MP_MAX_BLOCKS] = {}, *c1[MP_MAX_BLOCKS] = {}, *A2[MP_MAX_BLOCKS] = {},
+        *c2[MP_MAX_BLOCKS] = {};
+  float *W_in[MP_MAX_BLOCKS] = {}, *b_in[MP_MAX_BLOCKS] = {}, *W_out[MP_MAX_BLOCKS] = {},
+        *b_out[MP_MAX_BLOCKS] = {};
+  float *W_inT[MP_MAX_BLOCKS] = {}, *W_outT[MP_MAX_BLOCKS] = {};
+  float *B1 = nullptr, *d1 = nullptr, *B2 = nullptr, *d2 = nullptr, *B1T = nullptr;
+  float *Wq = nullptr, *Wk = nullptr, *P = nullptr, *p = nullptr;
+  // packed 16-bit operand images for the tensor-core kernels (see tc_*.cu)
+  void* tc_weights = nullptr;
+  size_t tc_weights_bytes = 0;
+  // workspace, sized from max_atoms
+  float* x_res = nullptr;                 // [N][F] fp32 residual stream
+  void* h[MP_MAX_BLOCKS] = {};            // [N][F] storage dtype: block inputs to the cfconv
+  void* m = nullptr;                      // [N][F] storage dtype: cfconv output
+  float* a = nullptr;                     // [N][F/2] readout pre-activation
+  float* u_ro = nullptr;                  // [N][F/2] readout backward
+  float* e_atom = nullptr;                // [N]
+  float* g_x = nullptr;                   // [N][F] dE/dx
+  void* g_m = nullptr;                    // [N][F] storage dtype: dE/dm
+  float* grad_h = nullptr;                // [N][F] dE/dh
+  float* q = nullptr;                     // [N][F] attention queries
+  float* k = nullptr;                     // [N][F] attention keys
+  int* status_d = nullptr;                // device status bits
+  int* status_h = nullptr;                // pinned host copy
+  long long launches = 0;
+  // profiling
+  bool profiling = false;
+  std::vector<cudaEvent_t> ev_pool;
+  std::vector<int> rec_kernel;            // kernel id per recorded pair
+  size_t rec_used = 0;
+  double prof_ms[mp::K_NUM] = {};
+  long long prof_n[mp::K_NUM] = {};
+  std::vector<int> prof_order;            // kernels seen, in first-seen order
+};
+
+namespace mp {
+
+// Launch a kernel, counting it and (when profiling) bracketing it with an event pair.
+template <typename Kern, typename... Args>
+inline int launch(mp_ctx* ctx, int kid, Kern kernel, dim3 grid, dim3 block, size_t smem,
+                  cudaStream_t s, Args... args) {
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  if (ctx && ctx->profiling && ctx->rec_used + 2 <= ctx->ev_pool.size()) {
+    e0 = ctx->ev_pool[ctx->rec_used];
+    e1 = ctx->ev_pool[ctx->rec_used + 1];
+    ctx->rec_used += 2;
+    ctx->rec_kernel.push_back(kid);
+    cudaEventRecord(e0, s);
+  }
+  kernel<<<grid, block, smem, s>>>(args...);
+  cudaError_t err = cudaGetLastError();
+  if (e1) cudaEventRecord(e1, s);
+  if (ctx) ctx->launches++;
+  return err == cudaSuccess ? MP_OK : MP_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Device helpers shared by the kernels.
+template <typename T>
+__device__ __forceinline__ float ldf(const T* p);
+template <>
+__device__ __forceinline__ float ldf<float>(const float* p) { return __ldg(p); }
+template <>
+__device__ __forceinline__ float ldf<__nv_bfloat16>(const __nv_bfloat16* p) {
+  return __bfloat162float(*p);
+}
+template <typename T>
+__device__ __forceinline__ void stf(T* p, float v);
+template <>
+__device__ __forceinline__ void stf<float>(float* p, float v) { *p = v; }
+template <>
+__device__ __forceinline__ void stf<__nv_bfloat16>(__nv_bfloat16* p, float v) {
+  *p = __float2bfloat16_rn(v);
+}
+
+// Shifted softplus ln(e^x/2 + 1/2) = max(x,0) + ln(1 + e^-|x|) - ln 2.
+__device__ __forceinline__ float ssp_f(float x) {
+  return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))) - 0.693147180559945309f;
+}
+__device__ __forceinline__ float sigmoid_f(float x) { return 1.f / (1.f + expf(-x)); }
+
+// Cosine envelope and its derivative; exactly 0 at and beyond the cutoff.
+__device__ __forceinline__ float cutoff_f(float d, float rc) {
+  return d < rc ? 0.5f * (cospif(d / rc) + 1.f) : 0.f;
+}
+__device__ __forceinline__ float cutoff_grad_f(float d, float rc) {
+  return d < rc ? -0.5f * 3.14159265358979f / rc * sinpif(d / rc) : 0.f;
+}
+
+__device__ __forceinline__ void raise_status(int* status, int bit) {
+  if (status) atomicOr(status, bit);
+}
+
+// Clamp a CSR offset read from device memory into [0, E].
+__device__ __forceinline__ long long clamp_off(long long v, long long E) {
+  return v < 0 ? 0 : (v > E ? E : v);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Host-side launchers implemented in the .cu files.
+int launch_embed(mp_ctx*, int N, const int* types, cudaStream_t);
+int launch_dense(mp_ctx*, int N, int Fin, int Fout, const void* in, bool in_bf16, const float* W,
+                 const float* b, bool residual, void* out, bool out_bf16, cudaStream_t);
+int launch_readout(mp_ctx*, int N, cudaStream_t);
+int launch_readout_bwd(mp_ctx*, int N, cudaStream_t);
+int launch_graph_sum(mp_ctx*, int N, const int* graph_ptr, int n_graphs, float* energy,
+                     cudaStream_t);
+int launch_cfconv_fwd_simt(mp_ctx*, int block, int N, long long E, const float* pos,
+                           const int* row_ptr, const int* col_idx, const void* x, void* out,
+                           cudaStream_t);
+int launch_cfconv_bwd_simt(mp_ctx*, int block, int N, long long E, const float* pos,
+                           const int* row_ptr, const int* col_idx, const void* h, const void* g,
+                           float* grad_h, float* forces, bool accumulate, cudaStream_t);
+int launch_attn_simt(mp_ctx*, int N, int K, const float* pos, const int* nbr,
+                     const unsigned char* mask, const void* x, void* out, cudaStream_t);
+int launch_validate_csr(mp_ctx*, int N, long long E, const int* row_ptr, const int* col_idx,
+                        const int* graph_ptr, int n_graphs, bool need_sym, cudaStream_t);
+
+FilterW filter_of(const mp_ctx* ctx, int block);
+Radial radial_of(const mp_ctx* ctx);
+
+}  // namespace mp

@@ -1,0 +1,434 @@
+"""Throughput of the fused message-passing path on B200.
+
+One step = one energy + forces evaluation (embedding, every interaction block's fused cfconv, readout,
+energy, and the fused backward giving forces) of the 10,000-atom workload (uniform at 0.1 atoms/A^3,
+cutoff 5 A, 3 blocks, F=128, 50 radial functions, bf16 storage with fp32 accumulation) with the
+neighbor list held fixed, through the library's public API. Inputs are resident in HBM when the timed
+region starts; the L2 cache is flushed (256 MiB write) between timed steps. Also reported: edges/s of
+one interaction block's cfconv, the end-to-end rate with host buffers (copies inside the timed region),
+the dominant kernel against its roofline, and the fp64 oracle on host cores as a CPU baseline.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference] [--workload cfg2]
+
+With N > 1 (launched by torchrun) every rank runs its own independent system (replicas, no collective
+on the data path): weak scaling; value = steps of all ranks / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "neighbor edges/sec per interaction block; MD steps/s (energy+forces) at 10k atoms"
+UNIT = "MD steps/s"
+FP32_LANES_PER_SM = 128  # FP32 FMA lanes per SM (B200)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--workload", default="cfg2")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-run", action="store_true",
+                    help="short run for ncu: no clocks sampler, no e2e, no CPU baseline")
+    return ap.parse_args()
+
+
+def rank_info():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "sm_max_mhz": d.get("sm_max_mhz", 1965.0), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------------------ clocks sampler
+class Clocks:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None, path: str):
+        self.path = path
+        self.proc = None
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "200"]
+        if gpu_id:
+            cmd += ["-i", gpu_id]
+        try:
+            self.f = open(path, "w")
+            self.proc = subprocess.Popen(cmd, stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append({"sm": float(parts[1]), "max": float(parts[2]),
+                             "power": float(parts[3]) if parts[3] not in ("[N/A]", "N/A") else 0.0,
+                             "hw": parts[5], "hwt": parts[6], "swt": parts[7], "pcap": parts[8]})
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        loaded = [r for r in rows if r["power"] > 150.0] or rows
+        reasons = set()
+        for r in loaded:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded),
+                "sm_max_mhz": max(r["max"] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows), "samples_under_load": len(loaded)}
+
+
+def gpu_uuid(torch, dev):
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------------------ work model
+def kernel_model(name: str, wl, E: int, N: int):
+    """(bound, algorithmic FLOPs or bytes per launch, unit) for a library kernel."""
+    R, F = wl.n_rbf, wl.F
+    fwd = 2.0 * (R * F + F * F) * E
+    if name == "cfconv_fwd_simt":
+        return "alu", fwd, "TFLOP/s"
+    if name == "cfconv_bwd_simt":
+        return "alu", 2.0 * fwd, "TFLOP/s"
+    if name == "cfconv_fwd_tc":
+        return "tensor", fwd, "TFLOP/s"
+    if name == "cfconv_bwd_tc":
+        return "tensor", 2.0 * fwd, "TFLOP/s"
+    if name == "dense":
+        return "hbm", (4 + 2 + 4) * N * F, "GB/s"
+    return "hbm", 0.0, "GB/s"
+
+
+def src_digest(kernel: str) -> str:
+    files = {"simt": "simt.cu", "tc": "tc_cfconv.cu"}
+    f = files["tc" if kernel.endswith("_tc") else "simt"]
+    data = open(os.path.join(ROOT, "atomistic_neighbor_list_b200", "csrc", f), "rb").read()
+    return hashlib.sha256(data).hexdigest()[:16]
+
+
+def traffic_for(kernel: str, units: int):
+    """DRAM bytes per launch from the committed ncu capture, if it is of the current source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(kernel)
+    if not d or d.get("src_sha") != src_digest(kernel):
+        return None
+    return d["dram_bytes_per_unit"] * units
+
+
+# ------------------------------------------------------------------------------ CPU baseline
+def cpu_baseline(wl, full_edges: int, budget_s: float):
+    """The fp64 oracle, as it stands, on a bounded same-density sample of the workload."""
+    import numpy as np
+
+    import oracle
+    from atomistic_neighbor_list_b200 import synth
+    w = synth.make_weights(wl)
+    model = oracle.Model.from_workload(wl, w)
+
+    def run(n):
+        sw = synth.scaled(wl, n)
+        pos, _ = synth.positions_for(sw)
+        types = synth.atom_types(n, wl.n_types)
+        rp, ci = oracle.neighbor_csr(pos, wl.r_c)
+        t = time.perf_counter()
+        oracle.energy_forces(model, pos, types, rp, ci)
+        return time.perf_counter() - t, len(ci)
+
+    t0, e0 = run(300)
+    n = int(min(wl.n_atoms, max(300, 300 * (budget_s / max(t0, 1e-3)) * 0.8)))
+    t1, e1 = (t0, e0) if n == 300 else run(n)
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    return {"value": (e1 / full_edges) / t1, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"one energy+forces step of a {n}-atom same-density system ({e1} edges, "
+                      f"{t1:.2f} s), scaled to the {full_edges}-edge workload by edge count",
+            "seconds": t1}
+
+
+def reference_arm(args):
+    rank, world, _ = rank_info()
+    if rank != 0:
+        return 0
+    from atomistic_neighbor_list_b200 import synth
+    import oracle
+    wl = synth.WORKLOADS[args.workload]
+    pos, _ = synth.positions_for(wl)
+    _, ci = oracle.neighbor_csr(pos, wl.r_c)
+    full_edges = len(ci)
+    budget = max(1.0, 150.0 / max(1, args.steps + args.warmup))
+    model = oracle.Model.from_workload(wl, synth.make_weights(wl))
+    # size the sample from a calibration step
+    def system(n):
+        sw = synth.scaled(wl, n)
+        p, _ = synth.positions_for(sw)
+        t = synth.atom_types(n, wl.n_types)
+        rp, c = oracle.neighbor_csr(p, wl.r_c)
+        return p, t, rp, c
+    p, t, rp, c = system(300)
+    s = time.perf_counter()
+    oracle.energy_forces(model, p, t, rp, c)
+    t300 = time.perf_counter() - s
+    n = int(min(wl.n_atoms, max(300, 300 * budget / max(t300, 1e-3) * 0.8)))
+    p, t, rp, c = system(n)
+    for _ in range(args.warmup):
+        oracle.energy_forces(model, p, t, rp, c)
+    times = []
+    for _ in range(args.steps):
+        s = time.perf_counter()
+        oracle.energy_forces(model, p, t, rp, c)
+        times.append(time.perf_counter() - s)
+    total = sum(times)
+    value = (len(c) / full_edges) * args.steps / total
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": 1000.0 / value, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+           "config": {"workload": wl.name, "atoms": wl.n_atoms, "edges": full_edges,
+                      "blocks": wl.n_blocks, "F": wl.F, "n_rbf": wl.n_rbf, "r_c": wl.r_c},
+           "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                            "sample": f"each step: energy+forces of a {n}-atom same-density "
+                                      f"system ({len(c)} edges), scaled by edge count"},
+           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------ main arm
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return reference_arm(args)
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from atomistic_neighbor_list_b200 import mp, synth
+
+    rank, world, local = rank_info()
+    torch.cuda.set_device(local)
+    devn = f"cuda:{local}"
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device(devn))
+    peaks = load_peaks()
+    wl = synth.WORKLOADS[args.workload]
+    pos, gp = synth.positions_for(wl, seed=rank)
+    N = len(pos)
+    types = synth.atom_types(N, wl.n_types)
+    weights = synth.make_weights(wl)
+    G = len(gp) - 1
+    pos_d = torch.from_numpy(pos).to(devn)
+    types_d = torch.from_numpy(types).to(devn)
+    gp_d = torch.from_numpy(gp).to(devn) if G > 1 else None
+    rp, ci = mp.neighbor_csr(pos_d, wl.r_c, graph_ptr=gp_d)
+    E = ci.numel()
+    ctx = mp.Context.from_workload(wl, weights, max_atoms=N, max_edges=E, max_graphs=G)
+    energy = torch.empty(G, dtype=torch.float32, device=devn)
+    forces = torch.empty((N, 3), dtype=torch.float32, device=devn)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=devn)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ctx.energy_forces(pos_d, types_d, rp, ci, gp_d, energy, forces)
+
+    clocks = None
+    if not args.profile_run:
+        clocks = Clocks(gpu_uuid(torch, local), os.path.join(ROOT, "gpurun_out",
+                                                               f"clocks_rank{rank}.csv")
+                        if os.path.isdir(os.path.join(ROOT, "gpurun_out"))
+                        else f"/tmp/mp_clocks_{os.getpid()}.csv")
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ctx.status_sync()
+
+    # ---- timed region: K steps, L2 flushed between steps, per-step CUDA events
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = ctx.launch_count()
+    ctx.profile_begin()
+    for k in range(args.steps):
+        flush.zero_()
+        evs[k][0].record(stream)
+        step()
+        evs[k][1].record(stream)
+    prof = ctx.profile_end()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    launches = ctx.launch_count() - launches0
+    total_ms = sum(a.elapsed_time(b) for a, b in evs)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=devn)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+    value = world * args.steps / (max_ms / 1000.0)
+
+    # ---- edges/s of one interaction block's cfconv (block 0), same timing rules
+    out_m = torch.empty((N, wl.F), dtype=torch.bfloat16 if wl.dtype == "bf16" else torch.float32,
+                        device=devn)
+    x_in = torch.from_numpy(synth.node_features(N, wl.F)).to(devn).to(out_m.dtype)
+    for _ in range(3):
+        ctx.cfconv_fwd(0, pos_d, rp, ci, x_in, out_m)
+    cf_ms = []
+    for _ in range(max(10, args.steps)):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        ctx.cfconv_fwd(0, pos_d, rp, ci, x_in, out_m)
+        b.record(stream)
+        cf_ms.append((a, b))
+    torch.cuda.synchronize()
+    cf_total = sum(a.elapsed_time(b) for a, b in cf_ms) / len(cf_ms)
+    edges_per_s = E / (cf_total / 1000.0)
+
+    # ---- end to end through the public API with host buffers (copies inside the timed region)
+    e2e = None
+    if not args.profile_run:
+        h_pos = torch.from_numpy(pos).pin_memory()
+        h_types = torch.from_numpy(types).pin_memory()
+        h_rp = rp.cpu().pin_memory()
+        h_ci = ci.cpu().pin_memory()
+        h_gp = torch.from_numpy(gp).pin_memory() if G > 1 else None
+        h_energy = torch.empty(G, dtype=torch.float32).pin_memory()
+        h_forces = torch.empty((N, 3), dtype=torch.float32).pin_memory()
+        d_pos, d_types = torch.empty_like(pos_d), torch.empty_like(types_d)
+        d_rp, d_ci = torch.empty_like(rp), torch.empty_like(ci)
+        d_gp = torch.empty_like(gp_d) if G > 1 else None
+
+        def e2e_step():
+            d_pos.copy_(h_pos, non_blocking=True)
+            d_types.copy_(h_types, non_blocking=True)
+            d_rp.copy_(h_rp, non_blocking=True)
+            d_ci.copy_(h_ci, non_blocking=True)
+            if G > 1:
+                d_gp.copy_(h_gp, non_blocking=True)
+            ctx.energy_forces(d_pos, d_types, d_rp, d_ci, d_gp, energy, forces)
+            h_energy.copy_(energy, non_blocking=True)
+            h_forces.copy_(forces, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        ev2 = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            e2e_step()
+            b.record(stream)
+            ev2.append((a, b))
+        torch.cuda.synchronize()
+        e2e_ms = torch.tensor([sum(a.elapsed_time(b) for a, b in ev2)], dtype=torch.float64,
+                              device=devn)
+        if world > 1:
+            dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+        bi = sum(x.numel() * x.element_size() for x in (h_pos, h_types, h_rp, h_ci)) + \
+            (h_gp.numel() * 4 if G > 1 else 0)
+        bo = h_energy.numel() * 4 + h_forces.numel() * 4
+        e2e = {"value": world * args.steps / (float(e2e_ms.item()) / 1000.0), "unit": UNIT,
+               "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo)}
+    ck = clocks.stop() if clocks else None
+    ctx.status_sync()
+
+    # ---- roofline of the dominant kernel (from the timed region's per-kernel events)
+    roofline = None
+    kernels = {}
+    if prof:
+        top = max(prof.items(), key=lambda kv: kv[1]["total_ms"])
+        name, st = top
+        avg_ms = st["total_ms"] / st["launches"]
+        bound, work, unit = kernel_model(name, wl, E, N)
+        if bound == "tensor":
+            peak = peaks["bf16_tflops_sustained"]
+            peak_note = f"{peaks['source']} bf16 sustained"
+        elif bound == "alu":
+            peak = 148 * FP32_LANES_PER_SM * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
+            peak_note = "FP32 FMA: 148 SMs x 128 lanes x 2 flop x max SM clock"
+        else:
+            peak = peaks["hbm_gbs"]
+            peak_note = f"{peaks['source']} HBM copy"
+        achieved = work / (avg_ms / 1000.0) / (1e12 if unit == "TFLOP/s" else 1e9)
+        traffic = traffic_for(name, E)
+        roofline = {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak,
+                    "unit": unit, "frac": achieved / peak, "traffic": traffic,
+                    "avg_launch_ms": avg_ms, "launches": st["launches"],
+                    "share_of_step": st["total_ms"] / max(total_ms, 1e-9),
+                    "peak_source": peak_note}
+        kernels = {k: {"ms_per_step": v["total_ms"] / args.steps,
+                       "launches_per_step": v["launches"] / args.steps} for k, v in prof.items()}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile_run:
+        cpu = cpu_baseline(wl, E, budget_s=15.0)
+
+    if rank == 0:
+        res = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+               "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
+               "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+               "dtype": wl.dtype, "data": "synthetic",
+               "config": {"workload": wl.name, "atoms": N, "edges": E, "blocks": wl.n_blocks,
+                          "F": wl.F, "n_rbf": wl.n_rbf, "r_c": wl.r_c, "graphs": G,
+                          "l2": "flushed between timed steps (256 MiB write)",
+                          "parallelism": f"replicas x{world} (independent systems, no collective)"},
+               "edges_per_s_per_block": {"value": edges_per_s, "unit": "edges/s",
+                                         "ms_per_block": cf_total},
+               "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+               "clocks": ck, "kernels": kernels}
+        print(json.dumps(res), flush=True)
+    ctx.close()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

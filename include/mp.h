@@ -1,0 +1,188 @@
+/*
+ * mp.h -- C ABI of libmp: fused neighbor-list message passing on NVIDIA B200 (sm_100a).
+ *
+ * The library computes, for SchNet-style atomistic force fields, the continuous-filter convolution
+ * over a destination-sorted CSR neighbor list (distance, Gaussian radial basis, cosine envelope,
+ * filter MLP, neighbor gather, filter product and segment sum fused in one pass, no atomics and no
+ * edge-by-feature tensor in memory), a neighbor attention aggregation with an online softmax over a
+ * padded neighbor list, and the energy with forces F = -dE/dr from a fused backward pass.
+ *
+ * Sources (page titles and sections):
+ *   [FS]  FlashSchNet: Fast and Accurate Coarse-Grained Neural Network Molecular Dynamics --
+ *         technical summary s.1 (bottlenecks), s.2.1 Flash Radial Basis, s.2.2 Flash Message Passing,
+ *         s.2.3 Flash Aggregation (CSR segment reduce by destination, by source in the backward),
+ *         s.2.4 channel-wise 16-bit quantization (positions, distances, energy accumulation and
+ *         forces stay fp32).
+ *   [E2]  E2Former-V2 page -- s.3.1 node-centric message passing, s.3.2 fused kernel (online softmax
+ *         with running maximum and normaliser, each key/value loaded once, padded neighbors masked,
+ *         parallel over destination atoms), s.5.2 (verify the neighbor list).
+ *   [TS]  Tessera page -- neighbor search and reuse, forces as the energy gradient.
+ *
+ * Conventions for every call:
+ *   - Array arguments are DEVICE pointers on the current CUDA device unless stated otherwise; the
+ *     caller owns them. Layouts are dense row-major. Positions are float32 [N][3] (Angstrom).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream) and is complete
+ *     only once that stream is synchronised. Calls do not synchronise, except where stated.
+ *   - Every call returns an mp_status. On any error no output is specified. Host-side argument
+ *     checks run before any launch. With mp_config.validate != 0 the CSR is also checked on the
+ *     device first (one stream synchronisation); a bad list returns MP_ERR_BAD_CSR /
+ *     MP_ERR_CSR_UNSORTED / MP_ERR_CSR_NOT_SYMMETRIC and nothing else runs. Compute kernels clamp
+ *     every index they read to the array bounds and raise MP_ERR_DEVICE_BOUNDS (reported by the
+ *     next mp_status_sync) instead of reading out of bounds.
+ *   - The CSR neighbor list: row_ptr int32 [N+1] with row_ptr[0] = 0 and row_ptr[N] = E,
+ *     col_idx int32 [E]; row i lists the sources j of edges j -> i, strictly ascending, j != i,
+ *     and no edge crosses a graph (replica). [FS s.2.3]
+ */
+#ifndef MP_H_
+#define MP_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MP_OK = 0,
+  MP_ERR_INVALID_ARG = -1,        /* null pointer, size out of range, unsupported configuration */
+  MP_ERR_BAD_CSR = -2,            /* row_ptr not monotone, wrong ends, or a column out of range */
+  MP_ERR_CSR_UNSORTED = -3,       /* a row not strictly ascending, or a self edge */
+  MP_ERR_CSR_NOT_SYMMETRIC = -4,  /* energy/forces need j in N(i) <=> i in N(j) */
+  MP_ERR_CAPACITY = -5,           /* N, E or a row exceeds what the context / output can hold */
+  MP_ERR_CUDA = -6,               /* a CUDA runtime call or launch failed */
+  MP_ERR_DEVICE_BOUNDS = -7,      /* a kernel met an index outside its arrays and skipped it */
+  MP_ERR_TIMEOUT = -8,            /* a bounded device wait ran out */
+  MP_ERR_UNIMPLEMENTED = -9
+} mp_status;
+
+typedef enum { MP_FP32 = 0, MP_BF16 = 1 } mp_dtype;
+
+#define MP_MAX_BLOCKS 8
+
+/* Model and capacity. Radial basis: e_k(d) = exp(-gamma (d - mu_k)^2), k = 0..n_rbf-1, with
+ * mu_k = mu_min + k (mu_max - mu_min)/(n_rbf - 1); envelope f_c(d) = (cos(pi d/r_c) + 1)/2 for
+ * d < r_c, else 0 [FS s.2.1]. Filter W(d) = f_c(d) (ssp(e(d) A1 + c1) A2 + c2) with
+ * ssp(x) = ln(e^x/2 + 1/2). Interaction block: h = x W_in + b_in; m = cfconv(h);
+ * x <- x + m W_out + b_out. Readout e_i = ssp(x_i B1 + d1) B2 + d2 (F -> F/2 -> 1).        */
+typedef struct {
+  int F;               /* channels: 64 or 128 */
+  int n_rbf;           /* radial functions, 2..64 */
+  int n_blocks;        /* interaction blocks, 1..MP_MAX_BLOCKS */
+  int n_types;         /* embedding rows (atom / bead types), >= 1 */
+  int n_heads;         /* attention heads; n_heads * head_dim == F */
+  int head_dim;
+  float r_c;           /* cutoff radius (Angstrom), > 0 */
+  float gamma;         /* Gaussian width parameter (1/Angstrom^2), > 0 */
+  float mu_min, mu_max;/* first and last radial centre */
+  mp_dtype dtype;      /* MP_FP32: fp32 features and math; MP_BF16: bf16 features and weights,
+                          fp32 accumulation; positions, distances, energy and forces fp32 [FS s.2.4] */
+  int max_atoms;       /* capacity of the internal workspace */
+  long long max_edges;
+  int max_graphs;      /* replicas per energy call */
+  int validate;        /* != 0: check the CSR on the device before each call */
+} mp_config;
+
+/* Weights: float32 row-major [in][out] arrays, host pointers (on_device = 0) or device pointers
+ * (on_device = 1). mp_init copies them (rounding to bf16, ties to even, under MP_BF16); the caller
+ * may free them after mp_init returns. Entries a call does not need may be NULL: energy/forces need
+ * emb, the first n_blocks entries of every per-block array and B1, d1, B2, d2; the cfconv needs
+ * A1, c1, A2, c2 of its block; the attention needs Wq, Wk, P, p and block 0's filter.       */
+typedef struct {
+  const float* emb;                       /* [n_types][F] */
+  const float* A1[MP_MAX_BLOCKS];         /* [n_rbf][F] */
+  const float* c1[MP_MAX_BLOCKS];         /* [F] */
+  const float* A2[MP_MAX_BLOCKS];         /* [F][F] */
+  const float* c2[MP_MAX_BLOCKS];         /* [F] */
+  const float* W_in[MP_MAX_BLOCKS];       /* [F][F] */
+  const float* b_in[MP_MAX_BLOCKS];       /* [F] */
+  const float* W_out[MP_MAX_BLOCKS];      /* [F][F] */
+  const float* b_out[MP_MAX_BLOCKS];      /* [F] */
+  const float* B1;                        /* [F][F/2] */
+  const float* d1;                        /* [F/2] */
+  const float* B2;                        /* [F/2][1] */
+  const float* d2;                        /* [1] */
+  const float* Wq;                        /* [F][F] attention query projection (no bias) */
+  const float* Wk;                        /* [F][F] attention key projection (no bias) */
+  const float* P;                         /* [n_rbf][n_heads] radial-basis logit bias */
+  const float* p;                         /* [n_heads] */
+  int on_device;
+} mp_weights;
+
+typedef struct mp_ctx mp_ctx;             /* opaque; one per device and model */
+
+/* Create a context on the current device: validates cfg, copies the weights, allocates the
+ * workspace (O(max_atoms * F * n_blocks) bytes, never O(E * F)). Synchronises `stream`.
+ * Errors: MP_ERR_INVALID_ARG, MP_ERR_CUDA.                                                  */
+int mp_init(mp_ctx** ctx, const mp_config* cfg, const mp_weights* w, void* stream);
+
+/* Release everything the context owns (synchronises the device first). NULL is ignored.     */
+void mp_destroy(mp_ctx* ctx);
+
+/* A static English description of a status code.                                           */
+const char* mp_strerror(int status);
+
+/* Synchronise `stream` and return (then clear) the device status word of the context:
+ * MP_OK, MP_ERR_DEVICE_BOUNDS or MP_ERR_CAPACITY raised by a kernel since the last call.    */
+int mp_status_sync(mp_ctx* ctx, void* stream);
+
+/* Neighbor list by the exact rule [FS s.2.3; E2 s.5.2; TS neighbor search]: j is a neighbor of
+ * i iff i != j, both in the same graph, and d2 < r_c*r_c, where d2 = (dx*dx + dy*dy) + dz*dz
+ * with (dx,dy,dz) = r_j - r_i, every step one correctly rounded float64 operation on the
+ * float32 positions (no fused multiply-add), r_c the float32 cutoff widened to float64.
+ * graph_ptr: int32 [n_graphs+1] contiguous atom ranges (device), or NULL for one graph.
+ * Output: row_ptr [N+1], col_idx [capacity] (device), rows sorted by source index.
+ * *n_edges (HOST pointer) receives E. Synchronises `stream` (to read E).
+ * Errors: MP_ERR_INVALID_ARG, MP_ERR_CAPACITY (E > capacity; row_ptr is valid, col_idx not). */
+int mp_neighbor_csr(int N, const float* pos, const int* graph_ptr, int n_graphs, float r_c,
+                    int* row_ptr, int* col_idx, long long capacity, long long* n_edges,
+                    void* stream);
+
+/* Fixed-width neighbor list for the attention aggregation [E2 s.3.2: padded neighbors are
+ * skipped by a mask]. Same rule as mp_neighbor_csr; a row with more than K neighbors keeps the
+ * K nearest by (d2, j); kept neighbors are stored by ascending j, then nbr = -1, mask = 0.
+ * nbr int32 [N][K], mask uint8 [N][K] (device). A row with more than 1024 candidates raises
+ * MP_ERR_CAPACITY (reported by the return value; synchronises `stream`).                      */
+int mp_neighbor_padded(int N, const float* pos, const int* graph_ptr, int n_graphs, float r_c,
+                       int K, int* nbr, unsigned char* mask, void* stream);
+
+/* One continuous-filter convolution [FS s.2.1-2.3] with block `block`'s filter weights:
+ *   out_i = sum_{j in row i} x_j (.) W(|r_i - r_j|),   rows with no edges give 0.
+ * x, out: [N][F] of the context dtype (float or bf16); out must not alias x. No atomics: each
+ * output row is written once. Errors: MP_ERR_INVALID_ARG, MP_ERR_CAPACITY, CSR errors (validate).*/
+int mp_cfconv_fwd(mp_ctx* ctx, int block, int N, long long E, const float* pos,
+                  const int* row_ptr, const int* col_idx, const void* x, void* out, void* stream);
+
+/* Neighbor attention aggregation with an online softmax [E2 s.3.1-3.2]. With q = x Wq,
+ * k = x Wk split into n_heads heads of head_dim channels, for each valid slot j of row i
+ * (mask != 0 and 0 <= nbr < N):
+ *   l_ijh = q_ih . k_jh / sqrt(head_dim) + sum_k e_k(d_ij) P_kh + p_h,
+ *   out_i[h] = sum_j softmax_j(l_ijh) (x_j (.) W(d_ij))[h]   (block 0's filter),
+ * a row with no valid slot gives 0. nbr int32 [N][K], mask uint8 [N][K], x/out [N][F] of the
+ * context dtype. Errors: MP_ERR_INVALID_ARG, MP_ERR_CAPACITY.                                */
+int mp_attn_fwd(mp_ctx* ctx, int N, int K, const float* pos, const int* nbr,
+                const unsigned char* mask, const void* x, void* out, void* stream);
+
+/* Energy and forces [FS s.1, s.2.3 backward by source; TS forces = -dE/dr]: embedding, n_blocks
+ * interaction blocks, readout; energy[g] = sum of atomic energies of graph g (fp32);
+ * forces [N][3] = -dE/dr (fp32) from the fused backward over the same CSR, which must be
+ * symmetric (true for any cutoff graph). types int32 [N] in [0, n_types); graph_ptr int32
+ * [n_graphs+1] (device) or NULL with n_graphs = 1. Errors: MP_ERR_INVALID_ARG,
+ * MP_ERR_CAPACITY, CSR errors (validate).                                                   */
+int mp_energy_forces(mp_ctx* ctx, int N, long long E, const float* pos, const int* types,
+                     const int* row_ptr, const int* col_idx, const int* graph_ptr, int n_graphs,
+                     float* energy, float* forces, void* stream);
+
+/* Kernel timing for measurement. mp_profile_begin makes later calls record a CUDA event pair
+ * around every kernel they launch (on the caller's stream); mp_profile_end synchronises the
+ * stream and folds the pairs into per-kernel totals, readable by index with mp_profile_get
+ * (name: static string; returns MP_ERR_INVALID_ARG past the last kernel).                   */
+int mp_profile_begin(mp_ctx* ctx);
+int mp_profile_end(mp_ctx* ctx, void* stream);
+int mp_profile_get(mp_ctx* ctx, int index, const char** name, double* total_ms,
+                   long long* launches);
+
+/* Number of kernels this context has launched since mp_init.                               */
+long long mp_launch_count(mp_ctx* ctx);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MP_H_ */

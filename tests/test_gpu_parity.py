@@ -1,0 +1,299 @@
+"""CUDA path vs the fp64 oracle, through the C-ABI, on seeded inputs of the five workloads.
+
+Neighbor lists and indices are compared bit for bit. Features: normwise max|d|/max|ref| <= 1e-5 on
+the fp32 path and <= 2e-2 on the bf16 path; forces: relative RMS <= 1e-2 on the bf16 path. The bf16
+oracle is the same fp64 code fed the bf16-rounded inputs and weights the library holds, so only the
+CUDA path's own intermediate roundings are measured. Full-size workloads are compared on sampled
+rows the oracle computes one by one, and through properties that hold at any size.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from atomistic_neighbor_list_b200 import synth
+from helpers import (TOL_BF16_FEAT, TOL_BF16_FORCE, TOL_FP32, features_for, normwise,
+                     oracle_weights, rel_rms)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def mp(cuda_ok):
+    from atomistic_neighbor_list_b200 import mp as _mp
+    return _mp
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+
+
+def make_ctx(mp, wl, weights, N, E, max_graphs=1, validate=False, dtype=None):
+    if dtype is not None:
+        import dataclasses
+        wl = dataclasses.replace(wl, dtype=dtype)
+    return mp.Context.from_workload(wl, weights, max_atoms=max(N, 1), max_edges=max(E, 1),
+                                    max_graphs=max_graphs, validate=validate), wl
+
+
+# ----------------------------------------------------------------------------- neighbor lists
+@pytest.mark.parametrize("key,n", [("cfg1", 512), ("cfg1", 1), ("cfg1", 2), ("cfg1", 777),
+                                   ("cfg2", 10_000), ("cfg5", 100_000)])
+def test_neighbor_csr_bit_exact(mp, key, n):
+    wl = synth.WORKLOADS[key]
+    pos = synth.uniform_positions(n, seed=0)
+    rp, ci = mp.neighbor_csr(dev(pos), wl.r_c)
+    orp, oci = oracle.neighbor_csr(pos, wl.r_c)
+    assert np.array_equal(rp.cpu().numpy(), orp)
+    assert np.array_equal(ci.cpu().numpy(), oci)
+
+
+def test_neighbor_csr_chains_bit_exact(mp):
+    wl = synth.WORKLOADS["cfg3"]
+    pos, gp = synth.positions_for(wl)
+    rp, ci = mp.neighbor_csr(dev(pos), wl.r_c, graph_ptr=dev(gp))
+    orp, oci = oracle.neighbor_csr(pos, wl.r_c, gp)
+    assert np.array_equal(rp.cpu().numpy(), orp)
+    assert np.array_equal(ci.cpu().numpy(), oci)
+
+
+def test_neighbor_csr_capacity_error(mp):
+    pos = synth.uniform_positions(300, seed=1)
+    with pytest.raises(mp.MpError) as e:
+        mp.neighbor_csr(dev(pos), 5.0, capacity=10)
+    assert e.value.name == "MP_ERR_CAPACITY"
+
+
+@pytest.mark.parametrize("n,K", [(600, 20), (32_768, 256)])
+def test_neighbor_padded_bit_exact(mp, n, K):
+    pos = synth.uniform_positions(n, seed=0)
+    nbr, mask = mp.neighbor_padded(dev(pos), 8.5 if K == 256 else 5.0, K)
+    onbr, omask = oracle.neighbor_padded(pos, 8.5 if K == 256 else 5.0, K)
+    assert np.array_equal(mask.cpu().numpy(), omask)
+    assert np.array_equal(nbr.cpu().numpy(), onbr)
+
+
+# ----------------------------------------------------------------------------- cfconv
+def cfconv_case(mp, key, n, dtype=None, rows=None, seed=0, block=0):
+    wl = synth.WORKLOADS[key]
+    if dtype:
+        import dataclasses
+        wl = dataclasses.replace(wl, dtype=dtype)
+    pos, gp = synth.positions_for(synth.scaled(wl, n) if wl.geometry == "uniform" else wl, seed)
+    n = len(pos)
+    w = synth.make_weights(wl)
+    rp, ci = mp.neighbor_csr(dev(pos), wl.r_c, graph_ptr=dev(gp) if len(gp) > 2 else None)
+    E = ci.numel()
+    ctx, wl = make_ctx(mp, wl, w, n, E)
+    x_t, x_ref = features_for(synth.node_features(n, wl.F), wl.dtype)
+    out = ctx.cfconv_fwd(block, dev(pos), rp, ci, x_t.to(DEV))
+    torch.cuda.synchronize()
+    ctx.status_sync()
+    model = oracle.Model.from_workload(wl, oracle_weights(w, wl.dtype))
+    ref = oracle.cfconv(model, block, pos, rp.cpu().numpy(), ci.cpu().numpy(), x_ref, rows=rows)
+    got = out.float().cpu().numpy().astype(np.float64)
+    if rows is not None:
+        got = got[rows]
+    return got, ref, ctx
+
+
+@pytest.mark.parametrize("n", [512, 1, 2, 37, 1000])
+def test_cfconv_fp32_cfg1(mp, n):
+    got, ref, _ = cfconv_case(mp, "cfg1", n)
+    assert normwise(got, ref) <= TOL_FP32
+
+
+@pytest.mark.parametrize("key,n", [("cfg2", 3000), ("cfg2", 10_000), ("cfg1", 512)])
+def test_cfconv_bf16(mp, key, n):
+    got, ref, _ = cfconv_case(mp, key, n, dtype="bf16")
+    assert normwise(got, ref) <= TOL_BF16_FEAT
+
+
+def test_cfconv_bf16_full_100k_sampled(mp):
+    rows = np.sort(np.random.default_rng(5).choice(100_000, 3000, replace=False))
+    got, ref, _ = cfconv_case(mp, "cfg5", 100_000, rows=rows)
+    assert normwise(got, ref) <= TOL_BF16_FEAT
+
+
+def test_cfconv_bf16_chains_sampled(mp):
+    rows = np.sort(np.random.default_rng(6).choice(64_000, 4000, replace=False))
+    got, ref, _ = cfconv_case(mp, "cfg3", 64_000, rows=rows, block=1)
+    assert normwise(got, ref) <= TOL_BF16_FEAT
+
+
+def test_cfconv_fp32_deterministic_and_empty_rows(mp):
+    wl = synth.WORKLOADS["cfg1"]
+    pos = synth.uniform_positions(300, seed=2)
+    pos[5] = [900.0, 900.0, 900.0]  # isolated atom: empty row
+    pos[299] = [-900.0, 0.0, 0.0]   # isolated last atom: empty trailing row
+    w = synth.make_weights(wl)
+    rp, ci = mp.neighbor_csr(dev(pos), wl.r_c)
+    ctx, _ = make_ctx(mp, wl, w, 300, ci.numel())
+    x = dev(synth.node_features(300, wl.F))
+    o1 = ctx.cfconv_fwd(0, dev(pos), rp, ci, x)
+    o2 = ctx.cfconv_fwd(0, dev(pos), rp, ci, x)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2)
+    assert torch.all(o1[5] == 0) and torch.all(o1[299] == 0)
+
+
+def test_cfconv_pair_at_exact_cutoff_is_zero(mp):
+    wl = synth.WORKLOADS["cfg1"]
+    w = synth.make_weights(wl)
+    # a hand-made CSR that includes a pair exactly at r_c: its message must be exactly zero
+    pos = np.array([[0, 0, 0], [5, 0, 0], [1, 1, 1]], dtype=np.float32)
+    rp = np.array([0, 1, 2, 2], dtype=np.int32)
+    ci = np.array([1, 0], dtype=np.int32)
+    ctx, _ = make_ctx(mp, wl, w, 3, 2)
+    out = ctx.cfconv_fwd(0, dev(pos), dev(rp), dev(ci), dev(synth.node_features(3, wl.F)))
+    torch.cuda.synchronize()
+    assert torch.all(out == 0)
+
+
+def test_cfconv_validate_rejects_bad_csr(mp):
+    wl = synth.WORKLOADS["cfg1"]
+    w = synth.make_weights(wl)
+    pos = synth.uniform_positions(50, seed=3)
+    rp, ci = mp.neighbor_csr(dev(pos), wl.r_c)
+    ctx, _ = make_ctx(mp, wl, w, 50, ci.numel() + 8, validate=True)
+    x = dev(synth.node_features(50, wl.F))
+    ctx.cfconv_fwd(0, dev(pos), rp, ci, x)  # valid list passes
+    bad = ci.clone()
+    bad[0] = 50  # column out of range
+    with pytest.raises(mp.MpError) as e:
+        ctx.cfconv_fwd(0, dev(pos), rp, bad, x)
+    assert e.value.name == "MP_ERR_BAD_CSR"
+    if rp[1].item() >= 2:
+        uns = ci.clone()
+        uns[0], uns[1] = ci[1].item(), ci[0].item()
+        with pytest.raises(mp.MpError) as e:
+            ctx.cfconv_fwd(0, dev(pos), rp, uns, x)
+        assert e.value.name == "MP_ERR_CSR_UNSORTED"
+    rp_bad = rp.clone()
+    rp_bad[-1] = rp_bad[-1] - 1
+    with pytest.raises(mp.MpError) as e:
+        ctx.cfconv_fwd(0, dev(pos), rp_bad, ci, x)
+    assert e.value.name == "MP_ERR_BAD_CSR"
+
+
+def test_cfconv_rejects_oversize(mp):
+    wl = synth.WORKLOADS["cfg1"]
+    w = synth.make_weights(wl)
+    ctx, _ = make_ctx(mp, wl, w, 10, 10)
+    pos = synth.uniform_positions(20, seed=3)
+    rp, ci = mp.neighbor_csr(dev(pos), wl.r_c)
+    with pytest.raises(mp.MpError) as e:
+        ctx.cfconv_fwd(0, dev(pos), rp, ci, dev(synth.node_features(20, wl.F)))
+    assert e.value.name == "MP_ERR_CAPACITY"
+
+
+# ----------------------------------------------------------------------------- attention
+def attn_case(mp, n, K, rows=None, dtype="bf16", r_c=8.5, seed=0):
+    import dataclasses
+    wl = dataclasses.replace(synth.WORKLOADS["cfg4"], n_atoms=n, K=K, dtype=dtype, r_c=r_c)
+    pos = synth.uniform_positions(n, seed=seed)
+    w = synth.make_weights(wl)
+    nbr, mask = mp.neighbor_padded(dev(pos), wl.r_c, K)
+    ctx, _ = make_ctx(mp, wl, w, n, 1)
+    x_t, x_ref = features_for(synth.node_features(n, wl.F), dtype)
+    out = ctx.attn_fwd(dev(pos), nbr, mask, x_t.to(DEV))
+    torch.cuda.synchronize()
+    ctx.status_sync()
+    model = oracle.Model.from_workload(wl, oracle_weights(w, dtype))
+    ref = oracle.attention(model, pos, nbr.cpu().numpy(), mask.cpu().numpy(), x_ref, rows=rows)
+    got = out.float().cpu().numpy().astype(np.float64)
+    return (got if rows is None else got[rows]), ref
+
+
+@pytest.mark.parametrize("n,K,dtype", [(700, 64, "fp32"), (700, 64, "bf16"), (2000, 256, "bf16"),
+                                       (33, 17, "fp32")])
+def test_attention_small(mp, n, K, dtype):
+    got, ref = attn_case(mp, n, K, dtype=dtype)
+    assert normwise(got, ref) <= (1e-5 if dtype == "fp32" else TOL_BF16_FEAT)
+
+
+def test_attention_full_32768_sampled(mp):
+    rows = np.sort(np.random.default_rng(7).choice(32_768, 600, replace=False))
+    got, ref = attn_case(mp, 32_768, 256, rows=rows)
+    assert normwise(got, ref) <= TOL_BF16_FEAT
+
+
+# ----------------------------------------------------------------------------- energy and forces
+def ef_case(mp, key, n=None, dtype=None, seed=0):
+    import dataclasses
+    wl = synth.WORKLOADS[key]
+    if dtype:
+        wl = dataclasses.replace(wl, dtype=dtype)
+    if n is not None and wl.geometry == "uniform":
+        wl = synth.scaled(wl, n)
+    pos, gp = synth.positions_for(wl, seed)
+    n = len(pos)
+    types = synth.atom_types(n, wl.n_types)
+    w = synth.make_weights(wl)
+    G = len(gp) - 1
+    rp, ci = mp.neighbor_csr(dev(pos), wl.r_c, graph_ptr=dev(gp) if G > 1 else None)
+    ctx, _ = make_ctx(mp, wl, w, n, ci.numel(), max_graphs=G)
+    E, F = ctx.energy_forces(dev(pos), dev(types), rp, ci, dev(gp) if G > 1 else None)
+    torch.cuda.synchronize()
+    ctx.status_sync()
+    model = oracle.Model.from_workload(wl, oracle_weights(w, wl.dtype))
+    Eref, Fref, e_atom = oracle.energy_forces(model, pos, types, rp.cpu().numpy(),
+                                              ci.cpu().numpy(), gp, return_atom_energy=True)
+    scale = np.array([np.abs(e_atom[gp[g]:gp[g + 1]]).sum() for g in range(G)])
+    return E.cpu().numpy().astype(np.float64), F.cpu().numpy().astype(np.float64), Eref, Fref, scale
+
+
+@pytest.mark.parametrize("key,n", [("fd64", 64), ("cfg5", 700), ("cfg1", 300)])
+def test_energy_forces_fp32(mp, key, n):
+    wl_key = key
+    E, F, Eref, Fref, scale = ef_case(mp, wl_key, n=n, dtype="fp32")
+    assert np.max(np.abs(E - Eref) / scale) <= 1e-5
+    assert rel_rms(F, Fref) <= 1e-4
+
+
+@pytest.mark.parametrize("key,n", [("fd64", 64), ("cfg2", 10_000)])
+def test_energy_forces_bf16(mp, key, n):
+    E, F, Eref, Fref, scale = ef_case(mp, key, n=n)
+    assert np.max(np.abs(E - Eref) / scale) <= TOL_BF16_FEAT
+    assert rel_rms(F, Fref) <= TOL_BF16_FORCE
+
+
+def test_energy_forces_bf16_replicas(mp):
+    E, F, Eref, Fref, scale = ef_case(mp, "cfg3")
+    assert E.shape == (64,)
+    assert np.max(np.abs(E - Eref) / scale) <= TOL_BF16_FEAT
+    assert rel_rms(F, Fref) <= TOL_BF16_FORCE
+
+
+def test_energy_forces_full_100k_properties(mp):
+    """100k atoms: net force ~ 0 and sampled forces vs the oracle on a cut-out sphere.
+
+    A force on atom k depends only on atoms within 2 * n_blocks * r_c of it, so the oracle on the
+    atoms within that radius (plus a margin) of a sampled atom gives that atom's exact force.
+    """
+    wl = synth.WORKLOADS["cfg5"]
+    pos, _ = synth.positions_for(wl)
+    n = len(pos)
+    types = synth.atom_types(n, wl.n_types)
+    w = synth.make_weights(wl)
+    rp, ci = mp.neighbor_csr(dev(pos), wl.r_c)
+    ctx, _ = make_ctx(mp, wl, w, n, ci.numel())
+    E, F = ctx.energy_forces(dev(pos), dev(types), rp, ci)
+    torch.cuda.synchronize()
+    ctx.status_sync()
+    F = F.cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(F)) and np.isfinite(E.item())
+    assert np.linalg.norm(F.sum(axis=0)) <= 1e-4 * np.linalg.norm(F, axis=1).sum()
+    centre = pos.mean(axis=0)
+    k = int(np.argmin(np.linalg.norm(pos - centre, axis=1)))
+    radius = 2 * wl.n_blocks * wl.r_c + 1.0
+    sel = np.nonzero(np.linalg.norm(pos - pos[k], axis=1) < radius)[0]
+    sub = pos[sel]
+    orp, oci = oracle.neighbor_csr(sub, wl.r_c)
+    model = oracle.Model.from_workload(wl, oracle_weights(w, wl.dtype))
+    _, Fsub = oracle.energy_forces(model, sub, types[sel], orp, oci)
+    kk = int(np.nonzero(sel == k)[0][0])
+    ref = Fsub[kk]
+    assert np.linalg.norm(F[k] - ref) <= 3e-2 * np.linalg.norm(ref)
