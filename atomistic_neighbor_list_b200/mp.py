@@ -65,6 +65,8 @@ def _load():
         "mp_profile_end": (i32, [vp, vp]),
         "mp_profile_get": (i32, [vp, i32, POINTER(c_char_p), POINTER(c_double), POINTER(i64)]),
         "mp_launch_count": (i64, [vp]),
+        "mp_attn_fwd_noalloc": (i32, [POINTER(MpConfig), POINTER(MpWeights), i32, i32, vp, vp, vp,
+                                      vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -77,7 +79,9 @@ lib = _load()
 
 EXPORTED = ("mp_init", "mp_destroy", "mp_strerror", "mp_status_sync", "mp_neighbor_csr",
             "mp_neighbor_padded", "mp_cfconv_fwd", "mp_attn_fwd", "mp_energy_forces",
-            "mp_profile_begin", "mp_profile_end", "mp_profile_get", "mp_launch_count")
+            "mp_profile_begin", "mp_profile_end", "mp_profile_get", "mp_launch_count",
+            "mp_attn_fwd_noalloc")
+NOALLOC_MAX_NF = 524288  # MP_NOALLOC_MAX_NF: largest N * F mp_attn_fwd_noalloc accepts
 
 
 def _check(status: int, what: str):
@@ -240,6 +244,38 @@ class Context:
             out[name.value.decode()] = {"total_ms": ms.value, "launches": n.value}
             i += 1
         return out
+
+
+def attn_fwd_noalloc(*, F: int, n_rbf: int, n_heads: int, head_dim: int, r_c: float,
+                     weights: dict, pos, nbr, mask, x, out=None, status=None, gamma: float = 10.0,
+                     mu_min: float = 0.0, mu_max: float | None = None, stream=None):
+    """mp_attn_fwd_noalloc: the fp32 attention aggregation with no context and no device allocation
+    inside the library. ``weights`` maps Wq, Wk, P, p, A1.0, c1.0, A2.0, c2.0 to float32 CUDA
+    tensors. The caller allocates ``out`` (and the optional int32 ``status`` tensor) beforehand."""
+    N, K = nbr.shape
+    _need(pos, "pos", torch.float32, (N, 3))
+    _need(nbr, "nbr", torch.int32, (N, K))
+    _need(mask, "mask", torch.uint8, (N, K))
+    _need(x, "x", torch.float32, (N, F))
+    if out is None:
+        out = torch.empty_like(x)
+    _need(out, "out", torch.float32, (N, F))
+    if status is not None:
+        _need(status, "status", torch.int32, (1,))
+    cfg = MpConfig(F=F, n_rbf=n_rbf, n_blocks=1, n_types=1, n_heads=n_heads, head_dim=head_dim,
+                   r_c=r_c, gamma=gamma, mu_min=mu_min, mu_max=r_c if mu_max is None else mu_max,
+                   dtype=FP32, max_atoms=N, max_edges=0, max_graphs=1, validate=0)
+    w = MpWeights()
+    for key in ("Wq", "Wk", "P", "p"):
+        setattr(w, key, ctypes.cast(_need(weights[key], key, torch.float32).data_ptr(), _FP))
+    for key in ("A1", "c1", "A2", "c2"):
+        getattr(w, key)[0] = ctypes.cast(_need(weights[f"{key}.0"], key, torch.float32).data_ptr(),
+                                         _FP)
+    w.on_device = 1
+    _check(lib.mp_attn_fwd_noalloc(ctypes.byref(cfg), ctypes.byref(w), N, K, _ptr(pos), _ptr(nbr),
+                                   _ptr(mask), _ptr(x), _ptr(out), _ptr(status), _stream(stream)),
+           "mp_attn_fwd_noalloc")
+    return out
 
 
 def neighbor_csr(pos, r_c: float, graph_ptr=None, capacity: int | None = None, stream=None):

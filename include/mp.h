@@ -160,6 +160,31 @@ int mp_cfconv_fwd(mp_ctx* ctx, int block, int N, long long E, const float* pos,
 int mp_attn_fwd(mp_ctx* ctx, int N, int K, const float* pos, const int* nbr,
                 const unsigned char* mask, const void* x, void* out, void* stream);
 
+/* Allocation-free attention aggregation (no counterpart in the paper; added for callers that
+ * cannot allocate device memory). Some hosts own every byte of device memory through their own
+ * pool or budget and hand a library only pre-allocated buffers -- an MD engine's plugin
+ * interface, a serving process under a fixed memory plan -- and a stray cudaMalloc (which can
+ * also synchronise the device) is not allowed there. mp_init allocates a workspace, so such
+ * callers use this entry point instead: it needs no context and calls no cudaMalloc, cudaFree or
+ * other allocating routine. It computes exactly what mp_attn_fwd computes on the fp32 path.
+ *   cfg: F, n_rbf, n_heads, head_dim, r_c, gamma, mu_min, mu_max are used; dtype must be MP_FP32.
+ *   w:   DEVICE pointers (on_device = 1) to fp32 Wq, Wk, P, p and A1[0], c1[0], A2[0], c2[0],
+ *        used as given (no copy, no rounding).
+ *   x, out: float32 [N][F] (device); status: optional device int that receives the kernel status
+ *        bits of this call (0 = fine; non-zero = an out-of-range neighbor index was skipped).
+ * Scratch: the query and key rows live in one static device array compiled into the library,
+ * 256 B + 8 * MP_NOALLOC_MAX_NF bytes (about 4 MiB) on every device that loads it, held until the
+ * process exits; N * F above MP_NOALLOC_MAX_NF returns MP_ERR_CAPACITY (N <= 4096 at F = 128).
+ * The first call on a device looks up the array's device address (once per device, with that
+ * device current); make that first call before any stream capture. Every call shares the array
+ * and it keeps the last call's contents: calls that overlap on the GPU (on different streams, or
+ * from different threads) race on it and must be serialised by the caller.
+ * Errors: MP_ERR_INVALID_ARG, MP_ERR_CAPACITY, MP_ERR_CUDA.                                    */
+#define MP_NOALLOC_MAX_NF 524288
+int mp_attn_fwd_noalloc(const mp_config* cfg, const mp_weights* w, int N, int K,
+                        const float* pos, const int* nbr, const unsigned char* mask,
+                        const float* x, float* out, int* status, void* stream);
+
 /* Energy and forces [FS s.1, s.2.3 backward by source; TS forces = -dE/dr]: embedding, n_blocks
  * interaction blocks, readout; energy[g] = sum of atomic energies of graph g (fp32);
  * forces [N][3] = -dE/dr (fp32) from the fused backward over the same CSR, which must be
