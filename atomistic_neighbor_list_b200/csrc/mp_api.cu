@@ -314,7 +314,7 @@ extern "C" int mp_energy_forces(mp_ctx* c, int N, long long E, const float* pos,
   }
   const int F = c->cfg.F, Fh = F / 2, B = c->cfg.n_blocks;
   const bool bf = c->cfg.dtype == MP_BF16;
-  const bool tc = tc_supported(c);
+  const bool tc = tc_supported(c), tc_bwd = tc_bwd_supported(c);
   int rc = MP_OK;
 #define MP_TRY(x)             \
   do {                        \
@@ -343,7 +343,7 @@ extern "C" int mp_energy_forces(mp_ctx* c, int N, long long E, const float* pos,
   MP_TRY(launch_dense(c, N, Fh, F, c->u_ro, false, c->B1T, nullptr, false, c->g_x, false, s));
   for (int b = B - 1; b >= 0; --b) {
     MP_TRY(launch_dense(c, N, F, F, c->g_x, false, c->W_outT[b], nullptr, false, c->g_m, bf, s));
-    if (tc)
+    if (tc_bwd)
       MP_TRY(tc_cfconv_bwd(c, b, N, E, pos, row_ptr, col_idx, c->h[b], c->g_m, c->grad_h, forces,
                            b != B - 1, s));
     else

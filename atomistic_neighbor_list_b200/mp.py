@@ -65,6 +65,7 @@ def _load():
         "mp_profile_end": (i32, [vp, vp]),
         "mp_profile_get": (i32, [vp, i32, POINTER(c_char_p), POINTER(c_double), POINTER(i64)]),
         "mp_launch_count": (i64, [vp]),
+        "mp_selftest_tc": (i32, [POINTER(i32)]),
         "mp_attn_fwd_noalloc": (i32, [POINTER(MpConfig), POINTER(MpWeights), i32, i32, vp, vp, vp,
                                       vp, vp, vp, vp]),
     }
@@ -80,7 +81,7 @@ lib = _load()
 EXPORTED = ("mp_init", "mp_destroy", "mp_strerror", "mp_status_sync", "mp_neighbor_csr",
             "mp_neighbor_padded", "mp_cfconv_fwd", "mp_attn_fwd", "mp_energy_forces",
             "mp_profile_begin", "mp_profile_end", "mp_profile_get", "mp_launch_count",
-            "mp_attn_fwd_noalloc")
+            "mp_attn_fwd_noalloc", "mp_selftest_tc")
 NOALLOC_MAX_NF = 524288  # MP_NOALLOC_MAX_NF: largest N * F mp_attn_fwd_noalloc accepts
 
 
@@ -276,6 +277,13 @@ def attn_fwd_noalloc(*, F: int, n_rbf: int, n_heads: int, head_dim: int, r_c: fl
                                    _ptr(mask), _ptr(x), _ptr(out), _ptr(status), _stream(stream)),
            "mp_attn_fwd_noalloc")
     return out
+
+
+def selftest_tc():
+    """Tensor-core layout self-check: returns the two mismatch counts (0, 0 when correct)."""
+    out = (c_int * 2)()
+    _check(lib.mp_selftest_tc(out), "mp_selftest_tc")
+    return int(out[0]), int(out[1])
 
 
 def neighbor_csr(pos, r_c: float, graph_ptr=None, capacity: int | None = None, stream=None):

@@ -207,6 +207,12 @@ int mp_profile_get(mp_ctx* ctx, int index, const char** name, double* total_ms,
 /* Number of kernels this context has launched since mp_init.                               */
 long long mp_launch_count(mp_ctx* ctx);
 
+/* Diagnostic: run the tensor-core layout self-check on the current device (one CTA; exact small-
+ * integer products through the shared-memory operand layouts the kernels use). mismatches (HOST,
+ * int[2]) receives the number of wrong outputs of the two checks (0 = pass; negative = an MMA did
+ * not complete within its bounded wait). Synchronises the device. Errors: MP_ERR_CUDA.       */
+int mp_selftest_tc(int* mismatches);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,110 @@
+"""Tensor-core (tcgen05) fused cfconv: layout self-check and the cases its tiling creates.
+
+A tile holds 128 edges in CSR order; rows longer than a tile are carried across tiles, a tile with
+more than 64 destination rows takes two segment-sum passes, rows without edges must come out zero.
+Each case is compared with the fp64 oracle fed the bf16 values the library holds.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from atomistic_neighbor_list_b200 import synth
+from helpers import TOL_BF16_FEAT, features_for, normwise, oracle_weights
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def mp(cuda_ok):
+    from atomistic_neighbor_list_b200 import mp as _mp
+    return _mp
+
+
+def test_layout_selftest(mp):
+    assert mp.selftest_tc() == (0, 0)
+
+
+def run_case(mp, pos, r_c=5.0, n_rbf=50, block=0, seed=0):
+    wl = dataclasses.replace(synth.WORKLOADS["cfg2"], n_atoms=len(pos), r_c=r_c, n_rbf=n_rbf,
+                             n_blocks=2)
+    w = synth.make_weights(wl, seed=seed + 2)
+    pos_d = torch.from_numpy(np.ascontiguousarray(pos, dtype=np.float32)).cuda()
+    rp, ci = mp.neighbor_csr(pos_d, r_c)
+    n = len(pos)
+    ctx = mp.Context.from_workload(wl, w, max_atoms=n, max_edges=max(ci.numel(), 1))
+    x_t, x_ref = features_for(synth.node_features(n, wl.F, seed=seed + 3), "bf16")
+    out = ctx.cfconv_fwd(block, pos_d, rp, ci, x_t.cuda())
+    torch.cuda.synchronize()
+    ctx.status_sync()
+    model = oracle.Model.from_workload(wl, oracle_weights(w, "bf16"))
+    ref = oracle.cfconv(model, block, pos, rp.cpu().numpy(), ci.cpu().numpy(), x_ref)
+    got = out.float().cpu().numpy()
+    return got, ref, rp.cpu().numpy()
+
+
+def test_rows_longer_than_a_tile(mp):
+    # r_c = 10 A at 0.1 atoms/A^3: about 400 neighbors per interior atom (3+ tiles per row)
+    pos = synth.uniform_positions(2500, seed=4)
+    got, ref, rp = run_case(mp, pos, r_c=10.0)
+    assert np.diff(rp).max() > 3 * 128
+    assert normwise(got, ref) <= TOL_BF16_FEAT
+
+
+def test_two_edges_per_row_two_segment_passes(mp):
+    # a straight line, spacing 4 A, cutoff 5 A: each row has at most 2 edges (64+ rows per tile)
+    n = 1000
+    pos = np.zeros((n, 3), dtype=np.float32)
+    pos[:, 0] = 4.0 * np.arange(n)
+    got, ref, rp = run_case(mp, pos)
+    assert np.diff(rp).max() == 2
+    assert normwise(got, ref) <= TOL_BF16_FEAT
+
+
+def test_one_edge_per_row_dimers_and_isolated(mp):
+    # dimers 3 A apart, dimers 50 A from each other, plus isolated atoms (empty rows)
+    rng = np.random.default_rng(0)
+    pos = []
+    for k in range(300):
+        base = np.array([50.0 * (k % 20), 50.0 * (k // 20), 0.0])
+        pos.append(base)
+        if k % 7 != 3:
+            pos.append(base + rng.normal(size=3) * 0.3 + np.array([3.0, 0, 0]))
+    pos.append(np.array([-500.0, 0, 0]))  # trailing empty row
+    pos = np.array(pos, dtype=np.float32)
+    got, ref, rp = run_case(mp, pos, seed=1)
+    assert np.diff(rp).min() == 0 and np.diff(rp).max() == 1
+    assert np.all(got[np.diff(rp) == 0] == 0)
+    assert normwise(got, ref) <= TOL_BF16_FEAT
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 37, 129, 700])
+def test_small_and_ragged(mp, n):
+    pos = synth.uniform_positions(n, seed=n)
+    got, ref, rp = run_case(mp, pos, seed=2)
+    if np.abs(ref).max() == 0:
+        assert np.all(got == 0)
+    else:
+        assert normwise(got, ref) <= TOL_BF16_FEAT
+
+
+def test_sixty_four_radial_functions(mp):
+    pos, _ = synth.chain_replicas(4, 300, seed=3)
+    got, ref, rp = run_case(mp, pos, r_c=10.0, n_rbf=64, block=1)
+    assert normwise(got, ref) <= TOL_BF16_FEAT
+
+
+def test_deterministic(mp):
+    wl = synth.WORKLOADS["cfg2"]
+    pos = synth.uniform_positions(5000, seed=9)
+    w = synth.make_weights(wl)
+    pos_d = torch.from_numpy(pos).cuda()
+    rp, ci = mp.neighbor_csr(pos_d, wl.r_c)
+    ctx = mp.Context.from_workload(wl, w, max_atoms=5000, max_edges=ci.numel())
+    x = torch.from_numpy(synth.node_features(5000, wl.F)).cuda().to(torch.bfloat16)
+    a = ctx.cfconv_fwd(0, pos_d, rp, ci, x)
+    b = ctx.cfconv_fwd(0, pos_d, rp, ci, x)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
