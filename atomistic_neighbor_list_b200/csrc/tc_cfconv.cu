@@ -19,41 +19,14 @@
 #include <cstring>
 #include <vector>
 
-#include "tc_api.cuh"
-#include "tc_ptx.cuh"
+#include "tc_common.cuh"
 
 namespace mp {
 namespace {
+using namespace tcc;
 
-constexpr int TM = 128;            // edges per tile
-constexpr int FT = 128;            // channels on this path
-constexpr int K2 = 128;            // second filter layer K
 constexpr int SLOT_PASS = 64;      // destination rows per segment-sum MMA
 constexpr int THREADS = 256;
-constexpr uint32_t WAIT_LIMIT = 1u << 22;
-constexpr float LOG2E = 1.4426950408889634f;
-constexpr float LN2 = 0.6931471805599453f;
-
-__host__ __device__ constexpr int k1_of(int R) { return ((R + 1) + 15) / 16 * 16; }
-
-// Byte offset of element (r, k) in a K-major no-swizzle operand whose K extent is kext.
-__host__ __device__ constexpr uint32_t kmaj(int r, int k, int kext) {
-  return (uint32_t)((r >> 3) * (kext * 16) + (k >> 3) * 128 + (r & 7) * 16 + (k & 7) * 2);
-}
-
-// Per-block packed weights: W1 [F][K1] (B operand of MMA1: W1[f][k] = A1[k][f], W1[f][R] = c1[f]),
-// W2 [F][128] (B operand of MMA2: W2[f][g] = A2[g][f]), c2 fp32 [F].
-struct ImgLayout {
-  size_t w1, w2, c2, bytes;
-};
-__host__ __device__ inline ImgLayout img_layout(int K1) {
-  ImgLayout L;
-  L.w1 = 0;
-  L.w2 = (size_t)FT * K1 * 2;
-  L.c2 = L.w2 + (size_t)FT * K2 * 2;
-  L.bytes = (L.c2 + FT * 4 + 1023) / 1024 * 1024;
-  return L;
-}
 
 // Shared-memory carve-up (offsets from a 1024-aligned base).
 struct Smem {
@@ -71,35 +44,6 @@ __host__ __device__ inline Smem smem_layout(int K1) {
   s.meta = s.c2 + FT * 4;
   s.total = s.meta + 6 * TM * 4 + 64;
   return s;
-}
-
-__device__ __forceinline__ float ssp_scaled(float z, float fc, float fcln2) {
-  // f_c * (max(z,0) + ln(1 + e^-|z|) - ln 2) = f_c max(z,0) + f_c ln2 log2((1 + e^-|z|) / 2)
-  const float t = tc::ex2f(-fabsf(z) * LOG2E);
-  const float l = tc::lg2f(fmaf(t, 0.5f, 0.5f));
-  return fmaf(fcln2, l, fc * fmaxf(z, 0.f));
-}
-
-__device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
-
-// largest r in [lo, hi) with row_ptr[r] <= e   (row_ptr nondecreasing; row_ptr[lo] <= e)
-__device__ __forceinline__ int row_of(const int* __restrict__ row_ptr, int lo, int hi, long long e) {
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if ((long long)row_ptr[mid] <= e) lo = mid; else hi = mid;
-  }
-  return lo;
-}
-
-// first r in [0, N] with row_ptr[r] >= v
-__device__ __forceinline__ int lower_row(const int* __restrict__ row_ptr, int N, long long v) {
-  int lo = 0, hi = N + 1;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if ((long long)row_ptr[mid] < v) lo = mid + 1; else hi = mid;
-  }
-  return lo;
 }
 
 __global__ void __launch_bounds__(THREADS, 2) k_cfconv_fwd_tc(
@@ -432,11 +376,11 @@ __global__ void __launch_bounds__(THREADS, 2) k_cfconv_fwd_tc(
 }  // namespace
 
 // ---------------------------------------------------------------------------------------------
+using namespace tcc;
+
 bool tc_supported(const mp_ctx* ctx) {
   return ctx->cfg.dtype == MP_BF16 && ctx->cfg.F == FT && ctx->tc_weights != nullptr;
 }
-
-bool tc_bwd_supported(const mp_ctx*) { return false; }
 
 int tc_prepare(mp_ctx* ctx, cudaStream_t s) {
   const mp_config& c = ctx->cfg;
@@ -495,10 +439,6 @@ int tc_cfconv_fwd(mp_ctx* ctx, int block, int N, long long E, const float* pos, 
                 ctx->status_d);
 }
 
-int tc_cfconv_bwd(mp_ctx*, int, int, long long, const float*, const int*, const int*, const void*,
-                  const void*, float*, float*, bool, cudaStream_t) {
-  return MP_ERR_UNIMPLEMENTED;
-}
 
 }  // namespace mp
 
@@ -509,6 +449,7 @@ int tc_cfconv_bwd(mp_ctx*, int, int, long long, const float*, const int*, const 
 // segment-sum MMA. Each thread checks one output row against a direct sum.
 namespace mp {
 namespace {
+using namespace tcc;
 
 __device__ __forceinline__ float st_a1(int m, int k) { return (float)(((m * 7 + k * 3) % 9) - 4); }
 __device__ __forceinline__ float st_b1(int n, int k) { return (float)(((n * 5 + k) % 7) - 3); }

@@ -108,3 +108,52 @@ def test_deterministic(mp):
     b = ctx.cfconv_fwd(0, pos_d, rp, ci, x)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+# ----------------------------------------------------------------------------- backward (forces)
+def run_ef(mp, pos, r_c=5.0, n_rbf=50, seed=0):
+    from helpers import TOL_BF16_FORCE, rel_rms
+    wl = dataclasses.replace(synth.WORKLOADS["cfg2"], n_atoms=len(pos), r_c=r_c, n_rbf=n_rbf,
+                             n_blocks=2)
+    w = synth.make_weights(wl, seed=seed + 2)
+    n = len(pos)
+    types = synth.atom_types(n, wl.n_types, seed=seed + 1)
+    pos_d = torch.from_numpy(np.ascontiguousarray(pos, dtype=np.float32)).cuda()
+    rp, ci = mp.neighbor_csr(pos_d, r_c)
+    ctx = mp.Context.from_workload(wl, w, max_atoms=n, max_edges=max(ci.numel(), 1))
+    E, F = ctx.energy_forces(pos_d, torch.from_numpy(types).cuda(), rp, ci)
+    torch.cuda.synchronize()
+    ctx.status_sync()
+    model = oracle.Model.from_workload(wl, oracle_weights(w, "bf16"))
+    Eref, Fref, e_atom = oracle.energy_forces(model, pos, types, rp.cpu().numpy(),
+                                              ci.cpu().numpy(), return_atom_energy=True)
+    e_err = abs(float(E[0]) - Eref[0]) / np.abs(e_atom).sum()
+    return e_err, rel_rms(F.cpu().numpy(), Fref), TOL_BF16_FORCE
+
+
+def test_forces_rows_longer_than_a_tile(mp):
+    e_err, f_err, tol = run_ef(mp, synth.uniform_positions(1500, seed=4), r_c=10.0)
+    assert e_err <= TOL_BF16_FEAT and f_err <= tol
+
+
+def test_forces_sparse_rows_and_empty_rows(mp):
+    n = 600
+    pos = np.zeros((n, 3), dtype=np.float32)
+    pos[:, 0] = 4.0 * np.arange(n)
+    pos[::50, 1] = 300.0  # every 50th atom isolated: empty rows
+    e_err, f_err, tol = run_ef(mp, pos, seed=1)
+    assert e_err <= TOL_BF16_FEAT and f_err <= tol
+
+
+@pytest.mark.parametrize("n", [2, 5, 130])
+def test_forces_small(mp, n):
+    pos = synth.uniform_positions(n, seed=n + 1)
+    pos = pos * (0.5 if n < 10 else 1.0)
+    e_err, f_err, tol = run_ef(mp, pos, seed=3)
+    assert e_err <= TOL_BF16_FEAT and f_err <= tol
+
+
+def test_forces_sixty_four_radial_functions(mp):
+    pos, _ = synth.chain_replicas(3, 250, seed=2)
+    e_err, f_err, tol = run_ef(mp, pos, r_c=10.0, n_rbf=64)
+    assert e_err <= TOL_BF16_FEAT and f_err <= tol
