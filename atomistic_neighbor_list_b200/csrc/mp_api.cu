@@ -14,7 +14,7 @@ const char* kernel_name(int id) {
   static const char* names[K_NUM] = {
       "embed", "dense", "readout_energy", "readout_bwd", "graph_energy_sum", "cfconv_fwd_simt",
       "cfconv_bwd_simt", "attn_simt", "validate_csr", "cfconv_fwd_tc", "cfconv_bwd_tc",
-      "attn_tc"};
+      "attn_tc", "dense_tc"};
   return (id >= 0 && id < K_NUM) ? names[id] : "?";
 }
 
@@ -89,6 +89,7 @@ void free_ctx(mp_ctx* c) {
   cudaDeviceSynchronize();
   cudaFree(c->emb);  // one allocation holds every weight array
   cudaFree(c->tc_weights);
+  cudaFree(c->tc_dense_img);
   cudaFree(c->x_res);  // one allocation holds the whole workspace
   cudaFree(c->status_d);
   if (c->status_h) cudaFreeHost(c->status_h);
@@ -321,6 +322,34 @@ extern "C" int mp_energy_forces(mp_ctx* c, int N, long long E, const float* pos,
     rc = (x);                 \
     if (rc != MP_OK) return rc; \
   } while (0)
+  if (tc && tc_bwd && N > 0) {
+    // bf16 path: every atomwise layer and both cfconv passes on the tensor cores
+    auto img = [&](int kind, int b) { return c->tc_dense_img + tc_dense_off(kind, b, B); };
+    MP_TRY(launch_embed(c, N, types, s));
+    for (int b = 0; b < B; ++b) {
+      MP_TRY(tc_dense(c, N, F, F, c->x_res, false, img(0, b), c->b_in[b], c->h[b], true,
+                      TC_DENSE_STORE, s));
+      MP_TRY(tc_cfconv_fwd(c, b, N, E, pos, row_ptr, col_idx, c->h[b], c->m, s));
+      MP_TRY(tc_dense(c, N, F, F, c->m, true, img(1, b), c->b_out[b], c->x_res, false,
+                      TC_DENSE_RESIDUAL, s));
+    }
+    // readout: pre-activation, atomic energies and dE/da in one pass
+    MP_TRY(tc_dense(c, N, F, Fh, c->x_res, false, img(4, 0), c->d1, c->u_ro, false,
+                    TC_DENSE_READOUT, s));
+    MP_TRY(launch_graph_sum(c, N, graph_ptr, n_graphs, energy, s));
+    MP_TRY(tc_dense(c, N, Fh, F, c->u_ro, false, img(5, 0), nullptr, c->g_x, false,
+                    TC_DENSE_STORE, s));
+    for (int b = B - 1; b >= 0; --b) {
+      MP_TRY(tc_dense(c, N, F, F, c->g_x, false, img(2, b), nullptr, c->g_m, true, TC_DENSE_STORE,
+                      s));
+      MP_TRY(tc_cfconv_bwd(c, b, N, E, pos, row_ptr, col_idx, c->h[b], c->g_m, c->grad_h, forces,
+                           b != B - 1, s));
+      if (b > 0)
+        MP_TRY(tc_dense(c, N, F, F, c->grad_h, false, img(3, b), nullptr, c->g_x, false,
+                        TC_DENSE_RESIDUAL, s));
+    }
+    return MP_OK;
+  }
   if (N > 0) {
     MP_TRY(launch_embed(c, N, types, s));
     for (int b = 0; b < B; ++b) {

@@ -34,7 +34,7 @@ struct FilterW {
 enum KernelId : int {
   K_EMBED = 0, K_DENSE, K_READOUT_E, K_READOUT_BWD, K_GRAPH_SUM, K_CFCONV_FWD_SIMT,
   K_CFCONV_BWD_SIMT, K_ATTN_SIMT, K_VALIDATE, K_CFCONV_FWD_TC, K_CFCONV_BWD_TC, K_ATTN_TC,
-  K_NUM
+  K_DENSE_TC, K_NUM
 };
 const char* kernel_name(int id);
 
@@ -56,6 +56,7 @@ struct mp_ctx {
   // packed 16-bit operand images for the tensor-core kernels (see tc_*.cu)
   void* tc_weights = nullptr;
   size_t tc_weights_bytes = 0;
+  uint8_t* tc_dense_img = nullptr;        // packed bf16 atomwise weights (tc_dense.cu)
   // workspace, sized from max_atoms
   float* x_res = nullptr;                 // [N][F] fp32 residual stream
   void* h[MP_MAX_BLOCKS] = {};            // [N][F] storage dtype: block inputs to the cfconv

@@ -11,7 +11,25 @@ bool tc_bwd_supported(const mp_ctx* ctx);
 int tc_prepare(mp_ctx* ctx, cudaStream_t s);
 int tc_cfconv_fwd(mp_ctx* ctx, int block, int N, long long E, const float* pos, const int* row_ptr,
                   const int* col_idx, const void* x, void* out, cudaStream_t s);
+// Warp-specialised pipelined variant of tc_cfconv_fwd (tc_cfconv_ws.cu).
+int tc_cfconv_fwd_ws(mp_ctx* ctx, int block, int N, long long E, const float* pos,
+                     const int* row_ptr, const int* col_idx, const void* x, void* out,
+                     cudaStream_t s);
 int tc_cfconv_bwd(mp_ctx* ctx, int block, int N, long long E, const float* pos, const int* row_ptr,
                   const int* col_idx, const void* h, const void* g, float* grad_h, float* forces,
                   bool accumulate, cudaStream_t s);
+// Atomwise layer on the tensor cores: out = in . W + b over rows (see tc_dense.cu for the modes).
+enum { TC_DENSE_STORE = 0, TC_DENSE_RESIDUAL = 1, TC_DENSE_READOUT = 2 };
+size_t tc_dense_bytes(int n_blocks);
+int tc_dense_pack(const float* W, int rows, int cols, bool transpose, uint8_t* dst);
+int tc_dense(mp_ctx* ctx, int N, int Kin, int Nout, const void* in, bool in_bf16,
+             const uint8_t* wimg, const float* bias, void* out, bool out_bf16, int mode,
+             cudaStream_t s);
+// Offsets of the packed dense images inside ctx->tc_dense_img.
+inline size_t tc_dense_off(int kind, int block, int n_blocks) {
+  // kind: 0 W_in, 1 W_out, 2 W_out^T, 3 W_in^T (per block), 4 B1, 5 B1^T
+  const size_t sq = (size_t)128 * 128 * 2;
+  if (kind < 4) return ((size_t)block * 4 + kind) * sq;
+  return (size_t)n_blocks * 4 * sq + (kind == 4 ? 0 : sq / 2);
+}
 }  // namespace mp

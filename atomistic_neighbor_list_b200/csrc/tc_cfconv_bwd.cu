@@ -26,17 +26,27 @@ constexpr int SLOT_PASS = 32;  // destination rows per segment-sum MMA
 struct SmemB {
   uint32_t w1, w2, x, y, c2, meta, total;
 };
-__host__ __device__ inline SmemB smem_layout_b(int K1) {
-  SmemB s;
-  s.w1 = 0;
-  s.w2 = s.w1 + FT * K1 * 2;
-  s.x = s.w2 + FT * K2 * 2;
-  const uint32_t xb = (uint32_t)(2 * TM * K1 * 2 > TM * K2 * 2 ? 2 * TM * K1 * 2 : TM * K2 * 2);
-  s.y = s.x + xb;
-  s.c2 = s.y + SLOT_PASS * TM * 2;
-  s.meta = s.c2 + FT * 4;
-  s.total = s.meta + 8192;
-  return s;
+__host__ __device__ constexpr uint32_t xbytes_b(int K1) {
+  return (uint32_t)(2 * TM * K1 * 2 > TM * K2 * 2 ? 2 * TM * K1 * 2 : TM * K2 * 2);
+}
+__host__ __device__ constexpr SmemB smem_layout_b(int K1) {
+  return SmemB{0u, (uint32_t)(FT * K1 * 2), (uint32_t)(FT * K1 * 2 + FT * K2 * 2),
+               (uint32_t)(FT * K1 * 2 + FT * K2 * 2) + xbytes_b(K1),
+               (uint32_t)(FT * K1 * 2 + FT * K2 * 2) + xbytes_b(K1) + SLOT_PASS * TM * 2,
+               (uint32_t)(FT * K1 * 2 + FT * K2 * 2) + xbytes_b(K1) + SLOT_PASS * TM * 2 + FT * 4,
+               (uint32_t)(FT * K1 * 2 + FT * K2 * 2) + xbytes_b(K1) + SLOT_PASS * TM * 2 + FT * 4 +
+                   9216};
+}
+
+__device__ __forceinline__ int dst_of_b(const int* __restrict__ s_rp, int r_lo, int r_end,
+                                        const int* __restrict__ row_ptr, long long g) {
+  if ((long long)s_rp[TM] <= g) return row_of(row_ptr, r_lo + TM, r_end, g);
+  int lo = 0, hi = TM;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if ((long long)s_rp[mid] <= g) lo = mid; else hi = mid;
+  }
+  return r_lo + lo;
 }
 
 __device__ __forceinline__ float rcpf(float x) {
@@ -45,14 +55,15 @@ __device__ __forceinline__ float rcpf(float x) {
   return r;
 }
 
+template <int K1>
 __global__ void __launch_bounds__(THREADS, 2) k_cfconv_bwd_tc(
     int N, long long E, const float* __restrict__ pos, const int* __restrict__ row_ptr,
     const int* __restrict__ col_idx, const __nv_bfloat16* __restrict__ hin,
     const __nv_bfloat16* __restrict__ gin, float* __restrict__ grad_h, float* __restrict__ forces,
-    int accumulate, const uint8_t* __restrict__ img, Radial rp, int K1, int* status) {
+    int accumulate, const uint8_t* __restrict__ img, Radial rp, int* status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  const SmemB L = smem_layout_b(K1);
+  constexpr SmemB L = smem_layout_b(K1);
   uint8_t* sW1 = sm + L.w1;
   uint8_t* sW2 = sm + L.w2;
   uint8_t* sX = sm + L.x;
@@ -70,10 +81,11 @@ __global__ void __launch_bounds__(THREADS, 2) k_cfconv_bwd_tc(
   int* s_slot_start = s_slot_row + TM;           // TM + 1 used
   float* s_part = (float*)(s_slot_start + TM + 4);  // [2][TM]
   float* s_force = s_part + 2 * TM;              // [TM][3]
-  int* s_wsum = (int*)(s_force + 3 * TM);        // 8
-  int* s_misc = s_wsum + 8;                      // 8
-  uint64_t* s_mbar = (uint64_t*)(s_misc + 8);
-  uint32_t* s_tmem = (uint32_t*)(s_mbar + 1);
+  int* s_rp = (int*)(s_force + 3 * TM);          // TM + 1 used (2 TM reserved)
+  int* s_wsum = s_rp + 2 * TM;                   // 8
+  int* s_misc = s_wsum + 8;                      // 8: nslots, -, r_begin, r_end, next r_lo
+  uint64_t* s_mbar = (uint64_t*)(s_misc + 8);    // [0] MMA completion, [1] weight copy
+  uint32_t* s_tmem = (uint32_t*)(s_mbar + 2);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, cta = blockIdx.x;
@@ -83,6 +95,7 @@ __global__ void __launch_bounds__(THREADS, 2) k_cfconv_bwd_tc(
     const int r1 = (cta == G - 1) ? N : lower_row(row_ptr, N, b_hi);
     s_misc[2] = r0;
     s_misc[3] = r1 > r0 ? r1 : r0;
+    s_misc[4] = r0;
   }
   __syncthreads();
   const int r_begin = s_misc[2], r_end = s_misc[3];
@@ -92,33 +105,29 @@ __global__ void __launch_bounds__(THREADS, 2) k_cfconv_bwd_tc(
   if (e_end < e_begin) e_end = e_begin;
 
   if (warp == 0) tc::tmem_alloc(s_tmem, 256);
-  if (tid == 0) tc::mbar_init(s_mbar, 1);
-  {
+  if (tid == 0) {
+    tc::mbar_init(&s_mbar[0], 1);
+    tc::mbar_init(&s_mbar[1], 1);
     const ImgLayout IL = img_layout(K1);
-    const uint4* g1 = (const uint4*)(img + IL.w1);
-    uint4* d1 = (uint4*)sW1;
-    for (int i = tid; i < FT * K1 * 2 / 16; i += THREADS) d1[i] = g1[i];
-    const uint4* g2 = (const uint4*)(img + IL.w2);
-    uint4* d2 = (uint4*)sW2;
-    for (int i = tid; i < FT * K2 * 2 / 16; i += THREADS) d2[i] = g2[i];
-    const float* gc2 = (const float*)(img + IL.c2);
-    for (int i = tid; i < FT; i += THREADS) sc2[i] = gc2[i];
+    tc::mbar_expect_tx(&s_mbar[1], FT * K1 * 2 + FT * K2 * 2 + FT * 4);
+    tc::bulk_g2s(sW1, img + IL.w1, FT * K1 * 2, &s_mbar[1]);
+    tc::bulk_g2s(sW2, img + IL.w2, FT * K2 * 2, &s_mbar[1]);
+    tc::bulk_g2s(sc2, img + IL.c2, FT * 4, &s_mbar[1]);
   }
-  tc::fence_proxy_async();
   tc::fence_before();
   __syncthreads();
   tc::fence_after();
   const uint32_t tmem = *s_tmem;
   const uint32_t idesc_ff = tc::idesc(TM, FT, 1, false, false);
   uint32_t phase = 0;
-  bool aborted = false;
+  bool aborted = __syncthreads_or(tc::mbar_wait(&s_mbar[1], 0, WAIT_LIMIT) ? 0 : 1) != 0;
 
   float carry = 0.f, fcarry = 0.f;
   int carry_row = -1;
   int next_row = r_begin;
 
   auto wait_mma = [&]() -> bool {
-    const int bad = tc::mbar_wait(s_mbar, phase, WAIT_LIMIT) ? 0 : 1;
+    const int bad = tc::mbar_wait(&s_mbar[0], phase, WAIT_LIMIT) ? 0 : 1;
     phase ^= 1u;
     tc::fence_after();
     return __syncthreads_or(bad) == 0;
@@ -143,16 +152,21 @@ __global__ void __launch_bounds__(THREADS, 2) k_cfconv_bwd_tc(
 
   for (long long tb = e_begin; tb < e_end && !aborted; tb += TM) {
     const int ne = (int)((e_end - tb) < TM ? (e_end - tb) : TM);
-    // ------------------------------------------------------------------ prep
+    const int r_lo = s_misc[4];
+    for (int i = tid; i <= TM; i += THREADS) s_rp[i] = row_ptr[min(r_lo + i, r_end)];
+    __syncthreads();
+    // ------------------------------------------------------------------ prep (all warps)
+    // half 0 writes the Gaussian row e, half 1 its d-derivative e'
     int my_dst = -1;
-    if (tid < TM) {
-      const int t = tid;
+    {
+      const int t = 32 * (warp & 3) + lane;
+      const int hf = warp >> 2;
       float fc = 0.f, dfc = 0.f, d = 0.f, ux = 0.f, uy = 0.f, uz = 0.f;
       int j = 0;
       bool ok = false;
       if (t < ne) {
         const long long gidx = tb + t;
-        my_dst = row_of(row_ptr, r_begin, r_end, gidx);
+        my_dst = dst_of_b(s_rp, r_lo, r_end, row_ptr, gidx);
         j = col_idx[gidx];
         if ((unsigned)j < (unsigned)N) {
           const float dx = pos[3 * my_dst] - pos[3 * j], dy = pos[3 * my_dst + 1] - pos[3 * j + 1],
@@ -168,43 +182,40 @@ __global__ void __launch_bounds__(THREADS, 2) k_cfconv_bwd_tc(
           }
           ok = true;
         } else {
-          raise_status(status, kStatusBounds);
+          if (hf == 0) raise_status(status, kStatusBounds);
           j = 0;
         }
       }
-      s_src[t] = j;
-      s_dst[t] = my_dst;
-      s_fc[t] = fc;
-      s_dfc[t] = dfc;
-      s_ux[t] = ux;
-      s_uy[t] = uy;
-      s_uz[t] = uz;
+      if (hf == 0) {
+        s_src[t] = j;
+        s_dst[t] = my_dst;
+        s_fc[t] = fc;
+        s_dfc[t] = dfc;
+        s_ux[t] = ux;
+        s_uy[t] = uy;
+        s_uz[t] = uz;
+      }
+      const float d0 = d - rp.mu_min;
+      uint8_t* dstA = sX + hf * (TM * K1 * 2);
+#pragma unroll
       for (int k0 = 0; k0 < K1; k0 += 8) {
-        uint32_t w[4], wd[4];
+        uint32_t w[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          float v[2], vd[2];
+          float v[2];
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             const int k = k0 + 2 * q + hh;
-            float val = 0.f, dval = 0.f;
-            if (ok) {
-              if (k < rp.R) {
-                const float dd = d - (rp.mu_min + k * rp.dmu);
-                val = tc::ex2f(nglog2e * dd * dd);
-                dval = -2.f * rp.gamma * dd * val;
-              } else if (k == rp.R) {
-                val = 1.f;  // bias column: z1 carries c1, t does not
-              }
-            }
-            v[hh] = val;
-            vd[hh] = dval;
+            const float dd = fmaf(-(float)k, rp.dmu, d0);
+            const float ek = tc::ex2f(nglog2e * dd * dd);
+            float val;
+            if (hf == 0) val = k < rp.R ? ek : (k == rp.R ? 1.f : 0.f);  // bias column: z1 only
+            else val = k < rp.R ? -2.f * rp.gamma * dd * ek : 0.f;
+            v[hh] = ok ? val : 0.f;
           }
           w[q] = tc::pack_bf16(v[0], v[1]);
-          wd[q] = tc::pack_bf16(vd[0], vd[1]);
         }
-        *(uint4*)(sX + kmaj(t, k0, K1)) = make_uint4(w[0], w[1], w[2], w[3]);
-        *(uint4*)(sX + TM * K1 * 2 + kmaj(t, k0, K1)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+        *(uint4*)(dstA + kmaj(t, k0, K1)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
     }
     __syncthreads();
@@ -234,6 +245,7 @@ __global__ void __launch_bounds__(THREADS, 2) k_cfconv_bwd_tc(
         s_misc[0] = ns;
         s_slot_start[ns] = ne;
       }
+      if (t == ne - 1) s_misc[4] = my_dst;  // the next tile starts in this row or later
     }
     __syncthreads();
     const int nslots = s_misc[0];
@@ -247,7 +259,7 @@ __global__ void __launch_bounds__(THREADS, 2) k_cfconv_bwd_tc(
       for (int ks = 0; ks < K1 / 16; ++ks)
         tc::mma(tmem + 128, tc::sdesc(sXe2_a + ks * 256, 128, K1 * 16),
                 tc::sdesc(sW1_a + ks * 256, 128, K1 * 16), idesc_ff, ks > 0);
-      tc::commit(s_mbar);
+      tc::commit(&s_mbar[0]);
     }
     if (!wait_mma()) {
       aborted = true;
@@ -290,7 +302,7 @@ __global__ void __launch_bounds__(THREADS, 2) k_cfconv_bwd_tc(
       for (int ks = 0; ks < K2 / 16; ++ks)
         tc::mma(tmem + 128, tc::sdesc(sX_a + ks * 256, 128, K2 * 16),
                 tc::sdesc(sW2_a + ks * 256, 128, K2 * 16), idesc_ff, ks > 0);
-      tc::commit(s_mbar);
+      tc::commit(&s_mbar[0]);
     }
     if (!wait_mma()) {
       aborted = true;
@@ -315,6 +327,22 @@ __global__ void __launch_bounds__(THREADS, 2) k_cfconv_bwd_tc(
         *(uint4*)(sX + kmaj(e, f0 + 8 * g8, K2)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
     }
+    // first 16-column chunk of the four gathered rows, loaded while MMA2a runs
+    const int j_me = s_src[e];
+    const int k_me = s_dst[e] >= 0 ? s_dst[e] : 0;
+    const uint4* gj = (const uint4*)(gin + (size_t)j_me * FT);
+    const uint4* hj = (const uint4*)(hin + (size_t)j_me * FT);
+    const uint4* gk = (const uint4*)(gin + (size_t)k_me * FT);
+    const uint4* hk = (const uint4*)(hin + (size_t)k_me * FT);
+    uint4 vgj[2], vhj[2], vgk[2], vhk[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int o = 8 * half + q;
+      vgj[q] = __ldg(gj + o);
+      vhj[q] = __ldg(hj + o);
+      vgk[q] = __ldg(gk + o);
+      vhk[q] = __ldg(hk + o);
+    }
     tc::fence_proxy_async();
     tc::fence_before();
     __syncthreads();
@@ -323,7 +351,7 @@ __global__ void __launch_bounds__(THREADS, 2) k_cfconv_bwd_tc(
       for (int ks = 0; ks < K2 / 16; ++ks)
         tc::mma(tmem, tc::sdesc(sX_a + ks * 256, 128, K2 * 16),
                 tc::sdesc(sW2_a + ks * 256, 128, K2 * 16), idesc_ff, ks > 0);
-      tc::commit(s_mbar);
+      tc::commit(&s_mbar[0]);
     }
     if (!wait_mma()) {
       aborted = true;
@@ -332,12 +360,6 @@ __global__ void __launch_bounds__(THREADS, 2) k_cfconv_bwd_tc(
     // ------------------------------------------------------------------ epi-2
     {
       const float fc = s_fc[e], dfc = s_dfc[e];
-      const int j = s_src[e];
-      const int k = s_dst[e] >= 0 ? s_dst[e] : 0;
-      const uint4* gj = (const uint4*)(gin + (size_t)j * FT);
-      const uint4* hj = (const uint4*)(hin + (size_t)j * FT);
-      const uint4* gk = (const uint4*)(gin + (size_t)k * FT);
-      const uint4* hk = (const uint4*)(hin + (size_t)k * FT);
       float s_acc = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -345,13 +367,23 @@ __global__ void __launch_bounds__(THREADS, 2) k_cfconv_bwd_tc(
         uint32_t ru[16], rv[16];
         tc::ld16(lane_base + f0, ru);
         tc::ld16(lane_base + 128 + f0, rv);
-        uint4 vgj[2], vhj[2], vgk[2], vhk[2];
+        float c2v[16];
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          vgj[q] = __ldg(gj + (f0 >> 3) + q);
-          vhj[q] = __ldg(hj + (f0 >> 3) + q);
-          vgk[q] = __ldg(gk + (f0 >> 3) + q);
-          vhk[q] = __ldg(hk + (f0 >> 3) + q);
+        for (int q = 0; q < 4; ++q) {
+          const float4 t4 = *(const float4*)(sc2 + f0 + 4 * q);
+          c2v[4 * q] = t4.x;
+          c2v[4 * q + 1] = t4.y;
+          c2v[4 * q + 2] = t4.z;
+          c2v[4 * q + 3] = t4.w;
+        }
+        if (c > 0) {
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            vgj[q] = __ldg(gj + (f0 >> 3) + q);
+            vhj[q] = __ldg(hj + (f0 >> 3) + q);
+            vgk[q] = __ldg(gk + (f0 >> 3) + q);
+            vhk[q] = __ldg(hk + (f0 >> 3) + q);
+          }
         }
         tc::ld_wait();
 #pragma unroll
@@ -368,7 +400,7 @@ __global__ void __launch_bounds__(THREADS, 2) k_cfconv_bwd_tc(
             for (int hh = 0; hh < 2; ++hh) {
               const int i = 8 * q + 2 * p2 + hh;
               const int f = f0 + i;
-              const float U = __uint_as_float(ru[i]) + sc2[f];
+              const float U = __uint_as_float(ru[i]) + c2v[i];
               const float Wv = fc * U;
               const float Wp = fmaf(dfc, U, fc * __uint_as_float(rv[i]));
               const float vgj_f = hh ? bf_hi(a_gj[p2]) : bf_lo(a_gj[p2]);
@@ -429,7 +461,7 @@ __global__ void __launch_bounds__(THREADS, 2) k_cfconv_bwd_tc(
         for (int ks = 0; ks < TM / 16; ++ks)
           tc::mma(tmem + p * SLOT_PASS, tc::sdesc(sX_a + ks * 256, 128, 2048),
                   tc::sdesc(sY_a + ks * 256, 128, TM * 16), id3, ks > 0);
-        tc::commit(s_mbar);
+        tc::commit(&s_mbar[0]);
       }
       if (!wait_mma()) {
         aborted = true;
@@ -476,7 +508,7 @@ __global__ void __launch_bounds__(THREADS, 2) k_cfconv_bwd_tc(
   if (aborted) {
     if (tid == 0) {
       raise_status(status, kStatusTimeout);
-      tc::mbar_wait(s_mbar, phase ^ 1u, WAIT_LIMIT);
+      tc::mbar_wait(&s_mbar[0], phase ^ 1u, WAIT_LIMIT);
     }
   } else if (tid < TM) {
     if (carry_row >= 0) write_row(carry_row, carry, fcarry);
@@ -498,18 +530,23 @@ int tc_cfconv_bwd(mp_ctx* ctx, int block, int N, long long E, const float* pos, 
                   const int* col_idx, const void* h, const void* g, float* grad_h, float* forces,
                   bool accumulate, cudaStream_t s) {
   const int K1 = k1_of(ctx->cfg.n_rbf);
-  const SmemB L = smem_layout_b(K1);
-  const size_t smem = L.total + 1024;
-  auto kern = k_cfconv_bwd_tc;
-  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   const ImgLayout IL = img_layout(K1);
   const uint8_t* img = (const uint8_t*)ctx->tc_weights + IL.bytes * block;
   long long tiles = (E + TM - 1) / TM;
   int grid = 2 * ctx->num_sms;
   if (tiles < grid) grid = (int)(tiles > 0 ? tiles : 1);
-  return launch(ctx, K_CFCONV_BWD_TC, kern, dim3(grid), dim3(THREADS), smem, s, N, E, pos, row_ptr,
-                col_idx, (const __nv_bfloat16*)h, (const __nv_bfloat16*)g, grad_h, forces,
-                (int)accumulate, img, radial_of(ctx), K1, ctx->status_d);
+  auto go = [&](auto kern, int k1) {
+    const size_t smem = smem_layout_b(k1).total + 1024;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    return launch(ctx, K_CFCONV_BWD_TC, kern, dim3(grid), dim3(THREADS), smem, s, N, E, pos,
+                  row_ptr, col_idx, (const __nv_bfloat16*)h, (const __nv_bfloat16*)g, grad_h,
+                  forces, (int)accumulate, img, radial_of(ctx), ctx->status_d);
+  };
+  if (K1 == 64) return go(k_cfconv_bwd_tc<64>, 64);
+  if (K1 == 80) return go(k_cfconv_bwd_tc<80>, 80);
+  if (K1 == 48) return go(k_cfconv_bwd_tc<48>, 48);
+  if (K1 == 32) return go(k_cfconv_bwd_tc<32>, 32);
+  return MP_ERR_INVALID_ARG;
 }
 
 }  // namespace mp

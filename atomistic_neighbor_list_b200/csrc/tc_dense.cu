@@ -1,0 +1,224 @@
+// Tensor-core (tcgen05 / TMEM) atomwise layers for the bf16 path: out = act(in . W + b) over 128-row
+// tiles, with the weight matrix held in shared memory as a packed bf16 operand and fp32 accumulation
+// in TMEM. The update network and the readout run in 16-bit on the tensor cores like the filter
+// (FlashSchNet page, technical summary s.2.4: W16A16 for the filter, update and readout networks;
+// energy accumulation in fp32).
+//
+// Epilogue modes (thread = row = TMEM lane):
+//   STORE     out[r] = acc + b              (bf16 or fp32)
+//   RESIDUAL  out[r] += acc + b             (fp32, in place)
+//   READOUT   a = acc + d1 (F/2 wide): e_atom[r] = sum_k ssp(a_k) B2_k + d2 and
+//             u[r][k] = sigmoid(a_k) B2_k = de_r/da_k, in one pass
+#include "tc_common.cuh"
+
+namespace mp {
+namespace {
+using namespace tcc;
+
+constexpr int DT = 128;  // rows per tile
+constexpr int DTHREADS = 128;
+
+enum { MODE_STORE = 0, MODE_RESIDUAL = 1, MODE_READOUT = 2 };
+
+struct DenseArgs {
+  int N, Kin, Nout;
+  const void* in;
+  int in_bf16;
+  const uint8_t* wimg;  // [Nout][Kin] bf16 K-major core-matrix layout
+  const float* bias;    // [Nout] or null
+  void* out;
+  int out_bf16;
+  int mode;
+  const float* B2;      // readout: [Nout]
+  const float* d2;      // readout: [1]
+  float* e_atom;        // readout: [N]
+};
+
+__global__ void __launch_bounds__(DTHREADS) k_dense_tc(DenseArgs a, int* status) {
+  // CTA = (row tile, 64-column slice of the output)
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sB = sm;                          // 64 x Kin bf16 (this CTA's output columns)
+  uint8_t* sA = sm + 64 * 128 * 2;           // 128 x Kin bf16
+  __shared__ uint64_t mbar_w, mbar;
+  __shared__ uint32_t tslot;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int Kin = a.Kin, nsplit = a.Nout / 64;
+  const int tile = blockIdx.x / nsplit, n0 = (blockIdx.x % nsplit) * 64;
+  if (warp == 0) tc::tmem_alloc(&tslot, 64);
+  if (tid == 0) {
+    tc::mbar_init(&mbar_w, 1);
+    tc::mbar_init(&mbar, 1);
+    const uint32_t wbytes = 64 * Kin * 2;
+    tc::mbar_expect_tx(&mbar_w, wbytes);
+    tc::bulk_g2s(sB, a.wimg + (size_t)n0 * Kin * 2, wbytes, &mbar_w);
+  }
+  const int r = tile * DT + tid;
+  const bool valid = r < a.N;
+  // ---- A tile: row r of the input, converted to bf16 (all loads of a half issued before use)
+  if (a.in_bf16) {
+    const uint4* src = (const uint4*)((const __nv_bfloat16*)a.in + (size_t)r * Kin);
+    uint4 v[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c)
+      v[c] = (valid && c < Kin / 8) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int c = 0; c < 16; ++c)
+      if (c < Kin / 8) *(uint4*)(sA + kmaj(tid, 8 * c, Kin)) = v[c];
+  } else {
+    const float4* src = (const float4*)((const float*)a.in + (size_t)r * Kin);
+#pragma unroll
+    for (int hb = 0; hb < 2; ++hb) {
+      if (hb * 64 >= Kin) break;
+      float4 v[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c)
+        v[c] = valid ? __ldg(src + hb * 16 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *(uint4*)(sA + kmaj(tid, hb * 64 + 8 * c, Kin)) =
+            make_uint4(tc::pack_bf16(v[2 * c].x, v[2 * c].y), tc::pack_bf16(v[2 * c].z, v[2 * c].w),
+                       tc::pack_bf16(v[2 * c + 1].x, v[2 * c + 1].y),
+                       tc::pack_bf16(v[2 * c + 1].z, v[2 * c + 1].w));
+    }
+  }
+  tc::fence_proxy_async();
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tmem = tslot;
+  int bad = 0;
+  if (tid == 0) {
+    if (!tc::mbar_wait(&mbar_w, 0, WAIT_LIMIT)) {
+      bad = 1;
+    } else {
+      const uint32_t sa = tc::smem_u32(sA), sb = tc::smem_u32(sB);
+      const uint32_t id = tc::idesc(DT, 64, 1, false, false);
+      for (int ks = 0; ks < Kin / 16; ++ks)
+        tc::mma(tmem, tc::sdesc(sa + ks * 256, 128, Kin * 16), tc::sdesc(sb + ks * 256, 128, Kin * 16),
+                id, ks > 0);
+      tc::commit(&mbar);
+    }
+  }
+  if (__syncthreads_or(bad)) {
+    if (tid == 0) raise_status(status, kStatusTimeout);
+  } else {
+    bad = tc::mbar_wait(&mbar, 0, WAIT_LIMIT) ? 0 : 1;
+    tc::fence_after();
+    if (__syncthreads_or(bad)) {
+      if (tid == 0) {
+        raise_status(status, kStatusTimeout);
+        tc::mbar_wait(&mbar, 0, WAIT_LIMIT);
+      }
+    } else {
+      // ---- epilogue: thread = row = TMEM lane, 64 columns
+      const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
+      float e_acc = 0.f;
+#pragma unroll
+      for (int c0 = 0; c0 < 64; c0 += 32) {
+        uint32_t rr[32];
+        tc::ld32(lane_base + c0, rr);
+        tc::ld_wait();
+        if (valid) {
+          const int col = n0 + c0;
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(rr[i]) + (a.bias ? a.bias[col + i] : 0.f);
+          if (a.mode == MODE_READOUT) {
+            float* u = (float*)a.out + (size_t)r * a.Nout + col;
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              float4 o;
+              float* po = &o.x;
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const float z = v[i + q], b2 = a.B2[col + i + q];
+                const float t = tc::ex2f(-fabsf(z) * LOG2E);
+                const float ssp = fmaf(LN2, tc::lg2f(fmaf(t, 0.5f, 0.5f)), fmaxf(z, 0.f));
+                e_acc = fmaf(ssp, b2, e_acc);
+                const float sg = z >= 0.f ? 1.f / (1.f + t) : t / (1.f + t);
+                po[q] = sg * b2;
+              }
+              *(float4*)(u + i) = o;
+            }
+          } else if (a.out_bf16) {
+            uint4* o = (uint4*)((__nv_bfloat16*)a.out + (size_t)r * a.Nout + col);
+#pragma unroll
+            for (int i = 0; i < 32; i += 8)
+              o[i / 8] = make_uint4(tc::pack_bf16(v[i], v[i + 1]), tc::pack_bf16(v[i + 2], v[i + 3]),
+                                    tc::pack_bf16(v[i + 4], v[i + 5]), tc::pack_bf16(v[i + 6], v[i + 7]));
+          } else {
+            float4* o = (float4*)((float*)a.out + (size_t)r * a.Nout + col);
+            float4 old[8];
+            if (a.mode == MODE_RESIDUAL) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) old[i] = o[i];
+            }
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              float4 w = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+              if (a.mode == MODE_RESIDUAL) {
+                w.x += old[i / 4].x;
+                w.y += old[i / 4].y;
+                w.z += old[i / 4].z;
+                w.w += old[i / 4].w;
+              }
+              o[i / 4] = w;
+            }
+          }
+        }
+      }
+      if (a.mode == MODE_READOUT && valid) a.e_atom[r] = e_acc + a.d2[0];
+    }
+  }
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem, 64);
+}
+
+}  // namespace
+
+// Packed dense weight images in ctx->tc_dense: per block W_in, W_out, W_out^T, W_in^T (each
+// [128][128]), then B1 ([64][128]) and B1^T ([128][64]).
+size_t tc_dense_bytes(int B) { return (size_t)(4 * B + 1) * 128 * 128 * 2; }
+
+int tc_dense_pack(const float* W, int rows, int cols, bool transpose, uint8_t* dst) {
+  // B operand [Nout][Kin]: element (n, k) = transpose ? W[n][k] : W[k][n], W row-major [rows][cols]
+  const int Nout = transpose ? rows : cols, Kin = transpose ? cols : rows;
+  for (int n = 0; n < Nout; ++n)
+    for (int k = 0; k < Kin; ++k) {
+      const float v = transpose ? W[(size_t)n * cols + k] : W[(size_t)k * cols + n];
+      uint32_t u;
+      memcpy(&u, &v, 4);
+      const uint16_t bits = (uint16_t)(u >> 16);  // values are bf16-rounded already
+      memcpy(dst + kmaj(n, k, Kin), &bits, 2);
+    }
+  return MP_OK;
+}
+
+int tc_dense(mp_ctx* ctx, int N, int Kin, int Nout, const void* in, bool in_bf16, const uint8_t* wimg,
+             const float* bias, void* out, bool out_bf16, int mode, cudaStream_t s) {
+  DenseArgs a;
+  a.N = N;
+  a.Kin = Kin;
+  a.Nout = Nout;
+  a.in = in;
+  a.in_bf16 = in_bf16;
+  a.wimg = wimg;
+  a.bias = bias;
+  a.out = out;
+  a.out_bf16 = out_bf16;
+  a.mode = mode;
+  a.B2 = ctx->B2;
+  a.d2 = ctx->d2;
+  a.e_atom = ctx->e_atom;
+  if (Nout % 64 != 0 || (Kin != 64 && Kin != 128) || (mode == MODE_READOUT && Nout != 64))
+    return MP_ERR_INVALID_ARG;
+  const size_t smem = 64 * 128 * 2 + 128 * 128 * 2 + 1024;
+  cudaFuncSetAttribute(k_dense_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const int ntiles = (N + DT - 1) / DT;
+  const int grid = (ntiles > 0 ? ntiles : 1) * (Nout / 64);
+  return launch(ctx, K_DENSE_TC, k_dense_tc, dim3(grid), dim3(DTHREADS), smem, s, a, ctx->status_d);
+}
+
+}  // namespace mp

@@ -93,6 +93,18 @@ __device__ __forceinline__ bool mbar_try(uint64_t* m, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of an mbarrier phase (for a thread that polls several barriers).
+__device__ __forceinline__ bool mbar_test(uint64_t* m, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n.reg .pred P1;\nmbarrier.test_wait.parity.shared::cta.b64 P1, [%1], %2;\n"
+      "selp.b32 %0, 1, 0, P1;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(m)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait on an mbarrier phase; false if the limit ran out.
 __device__ __forceinline__ bool mbar_wait(uint64_t* m, uint32_t parity, uint32_t limit) {
   for (uint32_t i = 0; i < limit; ++i)
@@ -100,8 +112,30 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* m, uint32_t parity, uint32_t
   return false;
 }
 
+// Expect `bytes` of asynchronous (TMA) traffic on the mbarrier and arrive once.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* m, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(m)),
+               "r"(bytes)
+               : "memory");
+}
+
+// One-dimensional bulk copy global -> this CTA's shared memory, completing on an mbarrier.
+// Addresses 16-byte aligned, size a multiple of 16. No multicast.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* m) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(m))
+      : "memory");
+}
+
 __device__ __forceinline__ void ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// 32 lanes x 32 bits, one column.
+__device__ __forceinline__ void ld1(uint32_t taddr, uint32_t& r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
 }
 
 // 32 lanes x 32 bits, 16 consecutive columns: thread t of the warp gets lane (base_lane + t).
