@@ -270,7 +270,8 @@ extern "C" int mp_cfconv_fwd(mp_ctx* c, int block, int N, long long E, const flo
                              const int* row_ptr, const int* col_idx, const void* x, void* out,
                              void* stream) {
   if (!c || block < 0 || block >= c->cfg.n_blocks || N < 0 || E < 0 || !row_ptr ||
-      (N > 0 && (!pos || !x || !out)) || (E > 0 && !col_idx) || (x && x == out))
+      (N > 0 && (!pos || !x || !out)) || (E > 0 && !col_idx) || (x && x == out) ||
+      ((uintptr_t)x & 15) != 0 || ((uintptr_t)out & 15) != 0)
     return MP_ERR_INVALID_ARG;
   if (N > c->cfg.max_atoms || E > c->cfg.max_edges) return MP_ERR_CAPACITY;
   cudaStream_t s = (cudaStream_t)stream;

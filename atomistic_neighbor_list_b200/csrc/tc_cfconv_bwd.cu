@@ -529,6 +529,13 @@ bool tc_bwd_supported(const mp_ctx* ctx) { return tc_supported(ctx); }
 int tc_cfconv_bwd(mp_ctx* ctx, int block, int N, long long E, const float* pos, const int* row_ptr,
                   const int* col_idx, const void* h, const void* g, float* grad_h, float* forces,
                   bool accumulate, cudaStream_t s) {
+  return tc_cfconv_bwd_ws(ctx, block, N, E, pos, row_ptr, col_idx, h, g, grad_h, forces, accumulate,
+                          s);
+}
+
+int tc_cfconv_bwd_sequential(mp_ctx* ctx, int block, int N, long long E, const float* pos,
+                             const int* row_ptr, const int* col_idx, const void* h, const void* g,
+                             float* grad_h, float* forces, bool accumulate, cudaStream_t s) {
   const int K1 = k1_of(ctx->cfg.n_rbf);
   const ImgLayout IL = img_layout(K1);
   const uint8_t* img = (const uint8_t*)ctx->tc_weights + IL.bytes * block;

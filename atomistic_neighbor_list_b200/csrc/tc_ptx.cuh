@@ -129,6 +129,32 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// TMA row gather: rows r0..r3 of a 2-D tensor map (columns c0 .. c0 + box width) into four
+// consecutive box rows of this CTA's shared memory, completing on an mbarrier. The map's box is one
+// row high; c0 times the element size is a multiple of 16 bytes. No multicast.
+__device__ __forceinline__ void tma_gather4(void* dst, const void* tmap, int c0, int r0, int r1,
+                                            int r2, int r3, uint64_t* m) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+      "l"(tmap), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(m))
+      : "memory");
+}
+
+// 16-byte asynchronous copy global -> shared (L2 only), and an arrival on an mbarrier once all of
+// this thread's earlier cp.async copies have landed (the arrival counts toward the expected count).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_arrive(uint64_t* m) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(m))
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 __device__ __forceinline__ void ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -136,6 +162,13 @@ __device__ __forceinline__ void ld_wait() {
 // 32 lanes x 32 bits, one column.
 __device__ __forceinline__ void ld1(uint32_t taddr, uint32_t& r) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+}
+
+// 32 lanes x 32 bits, 4 consecutive columns.
+__device__ __forceinline__ void ld4(uint32_t taddr, uint32_t (&r)[4]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr));
 }
 
 // 32 lanes x 32 bits, 16 consecutive columns: thread t of the warp gets lane (base_lane + t).

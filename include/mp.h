@@ -145,8 +145,10 @@ int mp_neighbor_padded(int N, const float* pos, const int* graph_ptr, int n_grap
 
 /* One continuous-filter convolution [FS s.2.1-2.3] with block `block`'s filter weights:
  *   out_i = sum_{j in row i} x_j (.) W(|r_i - r_j|),   rows with no edges give 0.
- * x, out: [N][F] of the context dtype (float or bf16); out must not alias x. No atomics: each
- * output row is written once. Errors: MP_ERR_INVALID_ARG, MP_ERR_CAPACITY, CSR errors (validate).*/
+ * x, out: [N][F] of the context dtype (float or bf16), 16-byte aligned (rows are read and
+ * written as 16-byte vectors); out must not alias x. No atomics: each output row is written once.
+ * Errors: MP_ERR_INVALID_ARG (also for a misaligned x or out), MP_ERR_CAPACITY, CSR errors
+ * (validate).                                                                                   */
 int mp_cfconv_fwd(mp_ctx* ctx, int block, int N, long long E, const float* pos,
                   const int* row_ptr, const int* col_idx, const void* x, void* out, void* stream);
 

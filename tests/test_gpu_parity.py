@@ -189,6 +189,30 @@ def test_cfconv_rejects_oversize(mp):
     assert e.value.name == "MP_ERR_CAPACITY"
 
 
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_cfconv_rejects_misaligned_rows(mp, dtype):
+    # x and out are read and written as 16-byte vectors: a pointer off that grid is refused on
+    # the host, before anything is launched
+    import dataclasses
+    wl = dataclasses.replace(synth.WORKLOADS["cfg1"], dtype=dtype)
+    w = synth.make_weights(wl)
+    n = 64
+    ctx, _ = make_ctx(mp, wl, w, n, 1)
+    pos = synth.uniform_positions(n, seed=4)
+    rp, ci = mp.neighbor_csr(dev(pos), wl.r_c)
+    tdt = torch.float32 if dtype == "fp32" else torch.bfloat16
+    flat = torch.zeros(n * wl.F + 1, dtype=tdt, device=DEV)
+    x_off = flat[1:].view(n, wl.F)
+    assert x_off.data_ptr() % 16 != 0
+    with pytest.raises(mp.MpError) as e:
+        ctx.cfconv_fwd(0, dev(pos), rp, ci, x_off)
+    assert e.value.name == "MP_ERR_INVALID_ARG"
+    x = torch.zeros(n, wl.F, dtype=tdt, device=DEV)
+    with pytest.raises(mp.MpError) as e:
+        ctx.cfconv_fwd(0, dev(pos), rp, ci, x, out=flat[1:].view(n, wl.F))
+    assert e.value.name == "MP_ERR_INVALID_ARG"
+
+
 # ----------------------------------------------------------------------------- attention
 def attn_case(mp, n, K, rows=None, dtype="bf16", r_c=8.5, seed=0):
     import dataclasses
