@@ -118,16 +118,14 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_cfconv_fwd_ws(
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, cta = blockIdx.x;
-  if (tid == 0) {
-    const long long b_lo = E * cta / G, b_hi = E * (cta + 1) / G;
-    const int r0 = lower_row(row_ptr, N, b_lo);
-    const int r1 = (cta == G - 1) ? N : lower_row(row_ptr, N, b_hi);
-    s_misc[8] = r0;
-    s_misc[9] = r1 > r0 ? r1 : r0;
-    s_misc[10] = 0;
+  if (warp < 2) {  // this CTA's rows: an edge-balanced split, both ends searched at once
+    const long long bnd = E * (cta + warp) / G;
+    const int r = (warp == 1 && cta == G - 1) ? N : warp_lower_row(row_ptr, N, bnd);
+    if (lane == 0) s_misc[8 + warp] = r;
+    if (tid == 0) s_misc[10] = 0;
   }
   __syncthreads();
-  const int r_begin = s_misc[8], r_end = s_misc[9];
+  const int r_begin = s_misc[8], r_end = max(s_misc[9], s_misc[8]);
   if (r_begin >= r_end) return;
   const long long e_begin = clamp_off(row_ptr[r_begin], E);
   long long e_end = clamp_off(row_ptr[r_end], E);

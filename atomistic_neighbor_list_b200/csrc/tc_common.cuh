@@ -111,6 +111,28 @@ __device__ __forceinline__ int lower_row(const int* __restrict__ row_ptr, int N,
   return lo;
 }
 
+// The same search by a whole warp (all 32 lanes call it): each round probes 32 rows at once, so
+// it takes ceil(log33(N + 1)) + 1 dependent loads instead of log2(N + 1). Result on every lane.
+__device__ __forceinline__ int warp_lower_row(const int* __restrict__ row_ptr, int N, long long v) {
+  const int lane = threadIdx.x & 31;
+  int lo = 0, hi = N + 1;  // the answer lies in [lo, hi); row_ptr[N] >= v for every v <= E
+  while (hi - lo > 32) {
+    const int len = hi - lo;
+    const int r = lo + (int)(((long long)len * (lane + 1)) / 33);
+    const unsigned hit = __ballot_sync(0xffffffffu, (long long)row_ptr[r] >= v);
+    if (hit == 0u) {
+      lo = lo + (int)(((long long)len * 32) / 33) + 1;
+    } else {
+      const int l = __ffs(hit) - 1;
+      hi = lo + (int)(((long long)len * (l + 1)) / 33) + 1;
+      if (l > 0) lo = lo + (int)(((long long)len * l) / 33) + 1;
+    }
+  }
+  const int r = lo + lane;
+  const unsigned hit = __ballot_sync(0xffffffffu, r < hi && (long long)row_ptr[r] >= v);
+  return hit ? lo + __ffs(hit) - 1 : hi;
+}
+
 
 }  // namespace tcc
 }  // namespace mp
