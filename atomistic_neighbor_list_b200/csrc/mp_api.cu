@@ -325,29 +325,30 @@ extern "C" int mp_energy_forces(mp_ctx* c, int N, long long E, const float* pos,
   } while (0)
   if (tc && tc_bwd && N > 0) {
     // bf16 path: every atomwise layer and both cfconv passes on the tensor cores
+    // consecutive atomwise layers that depend only on the row run as one launch (tc_dense2)
     auto img = [&](int kind, int b) { return c->tc_dense_img + tc_dense_off(kind, b, B); };
     MP_TRY(launch_embed(c, N, types, s));
-    for (int b = 0; b < B; ++b) {
-      MP_TRY(tc_dense(c, N, F, F, c->x_res, false, img(0, b), c->b_in[b], c->h[b], true,
-                      TC_DENSE_STORE, s));
-      MP_TRY(tc_cfconv_fwd(c, b, N, E, pos, row_ptr, col_idx, c->h[b], c->m, s));
-      MP_TRY(tc_dense(c, N, F, F, c->m, true, img(1, b), c->b_out[b], c->x_res, false,
-                      TC_DENSE_RESIDUAL, s));
-    }
-    // readout: pre-activation, atomic energies and dE/da in one pass
-    MP_TRY(tc_dense(c, N, F, Fh, c->x_res, false, img(4, 0), c->d1, c->u_ro, false,
-                    TC_DENSE_READOUT, s));
-    MP_TRY(launch_graph_sum(c, N, graph_ptr, n_graphs, energy, s));
-    MP_TRY(tc_dense(c, N, Fh, F, c->u_ro, false, img(5, 0), nullptr, c->g_x, false,
+    MP_TRY(tc_dense(c, N, F, F, c->x_res, false, img(0, 0), c->b_in[0], c->h[0], true,
                     TC_DENSE_STORE, s));
+    for (int b = 0; b < B; ++b) {
+      MP_TRY(tc_cfconv_fwd(c, b, N, E, pos, row_ptr, col_idx, c->h[b], c->m, s));
+      if (b + 1 < B)  // x += m W_out + b_out, then h of the next block = x W_in + b_in
+        MP_TRY(tc_dense2(c, N, F, c->m, true, img(1, b), c->b_out[b], c->x_res, TC_DENSE_RESIDUAL,
+                         img(0, b + 1), c->b_in[b + 1], F, c->h[b + 1], TC_DENSE_STORE, s));
+      else  // the last residual, then the readout: pre-activation, atomic energies and dE/da
+        MP_TRY(tc_dense2(c, N, F, c->m, true, img(1, b), c->b_out[b], c->x_res, TC_DENSE_RESIDUAL,
+                         img(4, 0), c->d1, Fh, c->u_ro, TC_DENSE_READOUT, s));
+    }
+    MP_TRY(launch_graph_sum(c, N, graph_ptr, n_graphs, energy, s));
+    // dE/dx = u B1^T, then g_m of the last block = dE/dx W_out^T
+    MP_TRY(tc_dense2(c, N, Fh, c->u_ro, false, img(5, 0), nullptr, c->g_x, TC_DENSE_STORE,
+                     img(2, B - 1), nullptr, F, c->g_m, TC_DENSE_STORE, s));
     for (int b = B - 1; b >= 0; --b) {
-      MP_TRY(tc_dense(c, N, F, F, c->g_x, false, img(2, b), nullptr, c->g_m, true, TC_DENSE_STORE,
-                      s));
       MP_TRY(tc_cfconv_bwd(c, b, N, E, pos, row_ptr, col_idx, c->h[b], c->g_m, c->grad_h, forces,
                            b != B - 1, s));
-      if (b > 0)
-        MP_TRY(tc_dense(c, N, F, F, c->grad_h, false, img(3, b), nullptr, c->g_x, false,
-                        TC_DENSE_RESIDUAL, s));
+      if (b > 0)  // dE/dx += grad_h W_in^T, then g_m of the block before = dE/dx W_out^T
+        MP_TRY(tc_dense2(c, N, F, c->grad_h, false, img(3, b), nullptr, c->g_x, TC_DENSE_RESIDUAL,
+                         img(2, b - 1), nullptr, F, c->g_m, TC_DENSE_STORE, s));
     }
     return MP_OK;
   }

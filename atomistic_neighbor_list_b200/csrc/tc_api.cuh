@@ -39,6 +39,12 @@ int tc_dense_pack(const float* W, int rows, int cols, bool transpose, uint8_t* d
 int tc_dense(mp_ctx* ctx, int N, int Kin, int Nout, const void* in, bool in_bf16,
              const uint8_t* wimg, const float* bias, void* out, bool out_bf16, int mode,
              cudaStream_t s);
+// Two dependent atomwise layers per 128-row tile (see tc_dense.cu): the first (STORE or RESIDUAL
+// into the fp32 out1), then the updated row through W2 (STORE as bf16 with N2 = 128, or READOUT
+// with N2 = 64).
+int tc_dense2(mp_ctx* ctx, int N, int K1, const void* in1, bool in1_bf16, const uint8_t* w1,
+              const float* b1, float* out1, int mode1, const uint8_t* w2, const float* b2, int N2,
+              void* out2, int mode2, cudaStream_t s);
 // Offsets of the packed dense images inside ctx->tc_dense_img.
 inline size_t tc_dense_off(int kind, int block, int n_blocks) {
   // kind: 0 W_in, 1 W_out, 2 W_out^T, 3 W_in^T (per block), 4 B1, 5 B1^T
