@@ -90,6 +90,7 @@ void free_ctx(mp_ctx* c) {
   cudaFree(c->emb);  // one allocation holds every weight array
   cudaFree(c->tc_weights);
   cudaFree(c->tc_dense_img);
+  cudaFree(c->tc_attn_p);
   cudaFree(c->x_res);  // one allocation holds the whole workspace
   cudaFree(c->status_d);
   if (c->status_h) cudaFreeHost(c->status_h);
@@ -297,6 +298,7 @@ extern "C" int mp_attn_fwd(mp_ctx* c, int N, int K, const float* pos, const int*
   int rc = launch_dense(c, N, F, F, x, bf, c->Wq, nullptr, false, c->q, false, s);
   if (rc == MP_OK) rc = launch_dense(c, N, F, F, x, bf, c->Wk, nullptr, false, c->k, false, s);
   if (rc != MP_OK) return rc;
+  if (tc_attn_supported(c, K)) return tc_attn_fwd(c, N, K, pos, nbr, mask, x, out, s);
   return launch_attn_simt(c, N, K, pos, nbr, mask, x, out, s);
 }
 

@@ -32,6 +32,11 @@ int tc_cfconv_bwd_ws(mp_ctx* ctx, int block, int N, long long E, const float* po
 int tc_cfconv_bwd(mp_ctx* ctx, int block, int N, long long E, const float* pos, const int* row_ptr,
                   const int* col_idx, const void* h, const void* g, float* grad_h, float* forces,
                   bool accumulate, cudaStream_t s);
+// Neighbor attention on the tensor cores (tc_attn.cu): 16 heads of 8, K a multiple of 128; q and
+// k (fp32 [N][F]) must already be in ctx->q, ctx->k.
+bool tc_attn_supported(const mp_ctx* ctx, int K);
+int tc_attn_fwd(mp_ctx* ctx, int N, int K, const float* pos, const int* nbr,
+                const unsigned char* mask, const void* x, void* out, cudaStream_t s);
 // Atomwise layer on the tensor cores: out = in . W + b over rows (see tc_dense.cu for the modes).
 enum { TC_DENSE_STORE = 0, TC_DENSE_RESIDUAL = 1, TC_DENSE_READOUT = 2 };
 size_t tc_dense_bytes(int n_blocks);

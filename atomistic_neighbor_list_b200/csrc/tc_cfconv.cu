@@ -453,6 +453,24 @@ int tc_prepare(mp_ctx* ctx, cudaStream_t s) {
     if (cudaMemcpy(ctx->tc_dense_img, dimg.data(), dimg.size(), cudaMemcpyHostToDevice) != cudaSuccess)
       return MP_ERR_CUDA;
   }
+  // attention (16 heads of 8): B rows 128..143 of its first MMA, P^T with the bias p on column R
+  if (c.n_heads == 16 && c.head_dim == 8 && ctx->P && ctx->p) {
+    const int H = c.n_heads;
+    std::vector<float> P((size_t)R * H), pb(H);
+    if (cudaMemcpy(P.data(), ctx->P, P.size() * 4, cudaMemcpyDeviceToHost) != cudaSuccess ||
+        cudaMemcpy(pb.data(), ctx->p, H * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+      return MP_ERR_CUDA;
+    std::vector<uint8_t> pimg((size_t)H * K1 * 2, 0);
+    for (int h = 0; h < H; ++h)
+      for (int k = 0; k < K1; ++k) {
+        const float v = k < R ? P[(size_t)k * H + h] : (k == R ? pb[h] : 0.f);
+        const uint16_t bits = bf16_bits(v);
+        std::memcpy(pimg.data() + kmaj(h, k, K1), &bits, 2);
+      }
+    if (cudaMalloc(&ctx->tc_attn_p, pimg.size()) != cudaSuccess ||
+        cudaMemcpy(ctx->tc_attn_p, pimg.data(), pimg.size(), cudaMemcpyHostToDevice) != cudaSuccess)
+      return MP_ERR_CUDA;
+  }
   if (cudaMalloc(&ctx->tc_weights, host.size()) != cudaSuccess) return MP_ERR_CUDA;
   ctx->tc_weights_bytes = host.size();
   if (cudaMemcpyAsync(ctx->tc_weights, host.data(), host.size(), cudaMemcpyHostToDevice, s) !=

@@ -345,6 +345,38 @@ def main():
     cf_total = sum(a.elapsed_time(b) for a, b in cf_ms) / len(cf_ms)
     edges_per_s = E / (cf_total / 1000.0)
 
+    # ---- attention variant (cfg4: 32,768 atoms, padded K = 256): edges/s counting valid edges,
+    # same timing rules; q and k projections included
+    attn = None
+    if not args.profile_run and rank == 0:
+        wl4 = synth.WORKLOADS["cfg4"]
+        pos4, _ = synth.positions_for(wl4, seed=0)
+        n4 = len(pos4)
+        pos4_d = torch.from_numpy(pos4).to(devn)
+        nbr4, mask4 = mp.neighbor_padded(pos4_d, wl4.r_c, wl4.K)
+        valid4 = int(mask4.sum().item())
+        ctx4 = mp.Context.from_workload(wl4, synth.make_weights(wl4), max_atoms=n4, max_edges=1)
+        x4 = torch.from_numpy(synth.node_features(n4, wl4.F)).to(devn).to(
+            torch.bfloat16 if wl4.dtype == "bf16" else torch.float32)
+        o4 = torch.empty_like(x4)
+        for _ in range(3):
+            ctx4.attn_fwd(pos4_d, nbr4, mask4, x4, o4)
+        ev4 = []
+        for _ in range(max(10, args.steps // 3)):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            ctx4.attn_fwd(pos4_d, nbr4, mask4, x4, o4)
+            b.record(stream)
+            ev4.append((a, b))
+        torch.cuda.synchronize()
+        ctx4.status_sync()
+        ms4 = sum(a.elapsed_time(b) for a, b in ev4) / len(ev4)
+        attn = {"value": valid4 / (ms4 / 1000.0), "unit": "edges/s", "ms_per_call": ms4,
+                "workload": f"cfg4 ({n4} atoms, K={wl4.K}, {valid4} valid edges, {wl4.dtype})"}
+        ctx4.close()
+        del nbr4, mask4, x4, o4, pos4_d
+
     # ---- end to end through the public API with host buffers (copies inside the timed region)
     e2e = None
     if not args.profile_run:
@@ -434,6 +466,7 @@ def main():
                           "F": wl.F, "n_rbf": wl.n_rbf, "r_c": wl.r_c, "graphs": G,
                           "l2": "flushed between timed steps (256 MiB write)",
                           "parallelism": f"replicas x{world} (independent systems, no collective)"},
+               "attention_edges_per_s": attn,
                "edges_per_s_per_block": {"value": edges_per_s, "unit": "edges/s",
                                          "ms_per_block": cf_total},
                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,

@@ -238,6 +238,36 @@ def test_attention_small(mp, n, K, dtype):
     assert normwise(got, ref) <= (1e-5 if dtype == "fp32" else TOL_BF16_FEAT)
 
 
+@pytest.mark.parametrize("n,K,r_c", [(1200, 128, 8.5), (3000, 384, 8.5), (1500, 256, 3.0)])
+def test_attention_tile_cases(mp, n, K, r_c):
+    # bf16, K a multiple of 128 (the tensor-core kernel): one tile per atom, three tiles merged
+    # by the running softmax, and a sparse cutoff where whole tiles (and some atoms) have no
+    # valid neighbor
+    got, ref = attn_case(mp, n, K, dtype="bf16", r_c=r_c)
+    assert np.isfinite(got).all()
+    assert normwise(got, ref) <= TOL_BF16_FEAT
+    if r_c < 4.0:
+        empty = np.abs(ref).max(axis=1) == 0.0
+        assert empty.any() and (got[empty] == 0.0).all()
+
+
+@pytest.mark.parametrize("K,kernel", [(256, "attn_tc"), (64, "attn_simt")])
+def test_attention_kernel_choice(mp, K, kernel):
+    # bf16 with K a multiple of 128 runs the tensor-core kernel, any other width the SIMT one
+    import dataclasses
+    wl = dataclasses.replace(synth.WORKLOADS["cfg4"], n_atoms=600, K=K, dtype="bf16")
+    pos = synth.uniform_positions(600, seed=2)
+    w = synth.make_weights(wl)
+    nbr, mask = mp.neighbor_padded(dev(pos), wl.r_c, K)
+    ctx, _ = make_ctx(mp, wl, w, 600, 1)
+    x = torch.from_numpy(synth.node_features(600, wl.F)).to(DEV).to(torch.bfloat16)
+    ctx.profile_begin()
+    ctx.attn_fwd(dev(pos), nbr, mask, x)
+    prof = ctx.profile_end()
+    assert kernel in prof and prof[kernel]["launches"] == 1
+    assert ({"attn_tc", "attn_simt"} - {kernel}).isdisjoint(prof)
+
+
 def test_attention_full_32768_sampled(mp):
     rows = np.sort(np.random.default_rng(7).choice(32_768, 600, replace=False))
     got, ref = attn_case(mp, 32_768, 256, rows=rows)
