@@ -91,6 +91,7 @@ void free_ctx(mp_ctx* c) {
   cudaFree(c->tc_weights);
   cudaFree(c->tc_dense_img);
   cudaFree(c->tc_attn_p);
+  if (c->ef_graph) cudaGraphExecDestroy(c->ef_graph);
   cudaFree(c->x_res);  // one allocation holds the whole workspace
   cudaFree(c->status_d);
   if (c->status_h) cudaFreeHost(c->status_h);
@@ -302,20 +303,10 @@ extern "C" int mp_attn_fwd(mp_ctx* c, int N, int K, const float* pos, const int*
   return launch_attn_simt(c, N, K, pos, nbr, mask, x, out, s);
 }
 
-extern "C" int mp_energy_forces(mp_ctx* c, int N, long long E, const float* pos, const int* types,
-                                const int* row_ptr, const int* col_idx, const int* graph_ptr,
-                                int n_graphs, float* energy, float* forces, void* stream) {
-  if (!c || N < 0 || E < 0 || !row_ptr || !energy || n_graphs < 1 ||
-      (N > 0 && (!pos || !types || !forces)) || (E > 0 && !col_idx) ||
-      (!graph_ptr && n_graphs != 1))
-    return MP_ERR_INVALID_ARG;
-  if (N > c->cfg.max_atoms || E > c->cfg.max_edges || n_graphs > c->cfg.max_graphs)
-    return MP_ERR_CAPACITY;
-  cudaStream_t s = (cudaStream_t)stream;
-  if (c->cfg.validate) {
-    int rc = launch_validate_csr(c, N, E, row_ptr, col_idx, graph_ptr, n_graphs, true, s);
-    if (rc != MP_OK) return rc;
-  }
+// The launches of one energy + forces evaluation (arguments already checked).
+static int energy_forces_launches(mp_ctx* c, int N, long long E, const float* pos, const int* types,
+                                  const int* row_ptr, const int* col_idx, const int* graph_ptr,
+                                  int n_graphs, float* energy, float* forces, cudaStream_t s) {
   const int F = c->cfg.F, Fh = F / 2, B = c->cfg.n_blocks;
   const bool bf = c->cfg.dtype == MP_BF16;
   const bool tc = tc_supported(c), tc_bwd = tc_bwd_supported(c);
@@ -387,6 +378,88 @@ extern "C" int mp_energy_forces(mp_ctx* c, int N, long long E, const float* pos,
                           s));
   }
 #undef MP_TRY
+  return MP_OK;
+}
+
+extern "C" int mp_energy_forces(mp_ctx* c, int N, long long E, const float* pos, const int* types,
+                                const int* row_ptr, const int* col_idx, const int* graph_ptr,
+                                int n_graphs, float* energy, float* forces, void* stream) {
+  if (!c || N < 0 || E < 0 || !row_ptr || !energy || n_graphs < 1 ||
+      (N > 0 && (!pos || !types || !forces)) || (E > 0 && !col_idx) ||
+      (!graph_ptr && n_graphs != 1))
+    return MP_ERR_INVALID_ARG;
+  if (N > c->cfg.max_atoms || E > c->cfg.max_edges || n_graphs > c->cfg.max_graphs)
+    return MP_ERR_CAPACITY;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (c->cfg.validate) {  // synchronises the stream to read its verdict: never captured
+    int rc = launch_validate_csr(c, N, E, row_ptr, col_idx, graph_ptr, n_graphs, true, s);
+    if (rc != MP_OK) return rc;
+  }
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  const bool use_graph = c->graphs && !c->graphs_broken && !c->profiling && !c->cfg.validate &&
+                         s != nullptr && cudaStreamIsCapturing(s, &cap) == cudaSuccess &&
+                         cap == cudaStreamCaptureStatusNone;
+  if (!use_graph)
+    return energy_forces_launches(c, N, E, pos, types, row_ptr, col_idx, graph_ptr, n_graphs,
+                                  energy, forces, s);
+  mp_ctx::EfKey key;
+  std::memset(&key, 0, sizeof key);  // padding included: the key is compared bytewise
+  key.N = N;
+  key.n_graphs = n_graphs;
+  key.E = E;
+  key.pos = pos;
+  key.types = types;
+  key.row_ptr = row_ptr;
+  key.col_idx = col_idx;
+  key.graph_ptr = graph_ptr;
+  key.energy = energy;
+  key.forces = forces;
+  key.stream = stream;
+  if (c->ef_graph && std::memcmp(&key, &c->ef_key, sizeof key) == 0) {  // a repeat: replay
+    if (cudaGraphLaunch(c->ef_graph, s) != cudaSuccess) return MP_ERR_CUDA;
+    c->launches += c->ef_launches;
+    return MP_OK;
+  }
+  if (c->ef_graph) {
+    cudaGraphExecDestroy(c->ef_graph);
+    c->ef_graph = nullptr;
+  }
+  // capture the launches once; on any failure fall back to plain launches for good
+  const long long l0 = c->launches;
+  cudaGraph_t g = nullptr;
+  int rc = cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal) == cudaSuccess ? MP_OK
+                                                                                     : MP_ERR_CUDA;
+  if (rc == MP_OK) {
+    rc = energy_forces_launches(c, N, E, pos, types, row_ptr, col_idx, graph_ptr, n_graphs, energy,
+                                forces, s);
+    if (cudaStreamEndCapture(s, &g) != cudaSuccess && rc == MP_OK) rc = MP_ERR_CUDA;
+  }
+  cudaGraphExec_t ex = nullptr;
+  if (rc == MP_OK && (!g || cudaGraphInstantiate(&ex, g, 0) != cudaSuccess)) rc = MP_ERR_CUDA;
+  if (g) cudaGraphDestroy(g);
+  const long long captured = c->launches - l0;  // kernels recorded into the graph (none ran)
+  c->launches = l0;
+  if (rc != MP_OK) {
+    cudaGetLastError();  // clear a capture error
+    c->graphs_broken = true;
+    return energy_forces_launches(c, N, E, pos, types, row_ptr, col_idx, graph_ptr, n_graphs,
+                                  energy, forces, s);
+  }
+  c->ef_graph = ex;
+  c->ef_key = key;
+  c->ef_launches = captured;
+  if (cudaGraphLaunch(ex, s) != cudaSuccess) return MP_ERR_CUDA;
+  c->launches += c->ef_launches;
+  return MP_OK;
+}
+
+extern "C" int mp_set_graphs(mp_ctx* c, int on) {
+  if (!c) return MP_ERR_INVALID_ARG;
+  c->graphs = on != 0;
+  if (!c->graphs && c->ef_graph) {
+    cudaGraphExecDestroy(c->ef_graph);
+    c->ef_graph = nullptr;
+  }
   return MP_OK;
 }
 

@@ -73,6 +73,16 @@ struct mp_ctx {
   int* status_d = nullptr;                // device status bits
   int* status_h = nullptr;                // pinned host copy
   long long launches = 0;
+  // CUDA graph of the last energy/forces call, replayed when a call repeats its arguments
+  bool graphs = true, graphs_broken = false;
+  cudaGraphExec_t ef_graph = nullptr;
+  long long ef_launches = 0;
+  struct EfKey {
+    int N, n_graphs;
+    long long E;
+    const void *pos, *types, *row_ptr, *col_idx, *graph_ptr;
+    void *energy, *forces, *stream;
+  } ef_key{};
   // profiling
   bool profiling = false;
   std::vector<cudaEvent_t> ev_pool;

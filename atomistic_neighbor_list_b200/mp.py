@@ -65,6 +65,7 @@ def _load():
         "mp_profile_end": (i32, [vp, vp]),
         "mp_profile_get": (i32, [vp, i32, POINTER(c_char_p), POINTER(c_double), POINTER(i64)]),
         "mp_launch_count": (i64, [vp]),
+        "mp_set_graphs": (i32, [vp, i32]),
         "mp_selftest_tc": (i32, [POINTER(i32)]),
         "mp_attn_fwd_noalloc": (i32, [POINTER(MpConfig), POINTER(MpWeights), i32, i32, vp, vp, vp,
                                       vp, vp, vp, vp]),
@@ -81,7 +82,7 @@ lib = _load()
 EXPORTED = ("mp_init", "mp_destroy", "mp_strerror", "mp_status_sync", "mp_neighbor_csr",
             "mp_neighbor_padded", "mp_cfconv_fwd", "mp_attn_fwd", "mp_energy_forces",
             "mp_profile_begin", "mp_profile_end", "mp_profile_get", "mp_launch_count",
-            "mp_attn_fwd_noalloc", "mp_selftest_tc")
+            "mp_attn_fwd_noalloc", "mp_selftest_tc", "mp_set_graphs")
 NOALLOC_MAX_NF = 524288  # MP_NOALLOC_MAX_NF: largest N * F mp_attn_fwd_noalloc accepts
 
 
@@ -232,6 +233,10 @@ class Context:
 
     def launch_count(self) -> int:
         return int(lib.mp_launch_count(self._ctx))
+
+    def set_graphs(self, on: bool):
+        """Record / replay energy_forces as a CUDA graph (default on; see mp_set_graphs)."""
+        _check(lib.mp_set_graphs(self._ctx, 1 if on else 0), "mp_set_graphs")
 
     def profile_begin(self):
         _check(lib.mp_profile_begin(self._ctx), "mp_profile_begin")

@@ -279,7 +279,10 @@ def main():
     energy = torch.empty(G, dtype=torch.float32, device=devn)
     forces = torch.empty((N, 3), dtype=torch.float32, device=devn)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=devn)
-    stream = torch.cuda.current_stream()
+    # a stream of its own, as an MD loop would run: the library records energy_forces as a CUDA
+    # graph on it and replays the graph every step (the legacy default stream cannot be captured)
+    stream = torch.cuda.Stream(device=devn)
+    torch.cuda.set_stream(stream)
 
     def step():
         ctx.energy_forces(pos_d, types_d, rp, ci, gp_d, energy, forces)
@@ -465,6 +468,7 @@ def main():
                "config": {"workload": wl.name, "atoms": N, "edges": E, "blocks": wl.n_blocks,
                           "F": wl.F, "n_rbf": wl.n_rbf, "r_c": wl.r_c, "graphs": G,
                           "l2": "flushed between timed steps (256 MiB write)",
+                          "launch": "energy_forces recorded once as a CUDA graph, replayed per step",
                           "parallelism": f"replicas x{world} (independent systems, no collective)"},
                "attention_edges_per_s": attn,
                "edges_per_s_per_block": {"value": edges_per_s, "unit": "edges/s",

@@ -197,6 +197,16 @@ int mp_energy_forces(mp_ctx* ctx, int N, long long E, const float* pos, const in
                      const int* row_ptr, const int* col_idx, const int* graph_ptr, int n_graphs,
                      float* energy, float* forces, void* stream);
 
+/* CUDA graphs for mp_energy_forces (on by default; a library addition, no counterpart on the
+ * pages). On a stream other than the legacy default stream, with profiling and validate off and
+ * no capture already in progress on it, a call records its kernels as a graph; a later call with
+ * the same N, E, n_graphs, array pointers and stream replays that graph (one launch), reading
+ * whatever the arrays hold then (new positions in the same buffer, for an MD step). A call with
+ * other arguments records a new graph in place of the old one. If recording fails, the call runs
+ * its kernels one by one and graphs stay off for the context. on = 0 turns graphs off and drops
+ * the recorded graph. Errors: MP_ERR_INVALID_ARG.                                            */
+int mp_set_graphs(mp_ctx* ctx, int on);
+
 /* Kernel timing for measurement. mp_profile_begin makes later calls record a CUDA event pair
  * around every kernel they launch (on the caller's stream); mp_profile_end synchronises the
  * stream and folds the pairs into per-kernel totals, readable by index with mp_profile_get
