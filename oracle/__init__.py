@@ -35,3 +35,4 @@ from .schnet import (  # noqa: F401
     ssp_grad, filter_weights, cfconv, Model, energies, energy_forces,
 )
 from .attention import attention  # noqa: F401
+from .md import kinetic_energy, velocity_verlet  # noqa: F401

@@ -40,3 +40,21 @@ def features_for(x: np.ndarray, dtype: str):
     if dtype == "bf16":
         t = t.to(torch.bfloat16)
     return t, t.float().numpy().astype(np.float64)
+
+
+def oracle_csr(pos, r_c: float, rp, ci, graph_ptr=None):
+    """The oracle's own cutoff CSR for the same positions, checked bit for bit against the CUDA
+    path's lists (rp, ci: torch tensors), which then serve the CUDA side only: every oracle input
+    comes from the seeded generator and the oracle itself."""
+    import oracle
+    orp, oci = oracle.neighbor_csr(pos, r_c, graph_ptr)
+    assert np.array_equal(rp.cpu().numpy(), orp) and np.array_equal(ci.cpu().numpy(), oci)
+    return orp, oci
+
+
+def oracle_padded(pos, r_c: float, K: int, nbr, mask):
+    """The oracle's own capped neighbor list, checked bit for bit against the CUDA path's."""
+    import oracle
+    onbr, omask = oracle.neighbor_padded(pos, r_c, K)
+    assert np.array_equal(mask.cpu().numpy(), omask) and np.array_equal(nbr.cpu().numpy(), onbr)
+    return onbr, omask

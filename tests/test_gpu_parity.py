@@ -13,7 +13,7 @@ import torch
 import oracle
 from atomistic_neighbor_list_b200 import synth
 from helpers import (TOL_BF16_FEAT, TOL_BF16_FORCE, TOL_FP32, features_for, normwise,
-                     oracle_weights, rel_rms)
+                     oracle_csr, oracle_padded, oracle_weights, rel_rms)
 
 pytestmark = pytest.mark.gpu
 
@@ -92,7 +92,8 @@ def cfconv_case(mp, key, n, dtype=None, rows=None, seed=0, block=0):
     torch.cuda.synchronize()
     ctx.status_sync()
     model = oracle.Model.from_workload(wl, oracle_weights(w, wl.dtype))
-    ref = oracle.cfconv(model, block, pos, rp.cpu().numpy(), ci.cpu().numpy(), x_ref, rows=rows)
+    orp, oci = oracle_csr(pos, wl.r_c, rp, ci, gp if len(gp) > 2 else None)
+    ref = oracle.cfconv(model, block, pos, orp, oci, x_ref, rows=rows)
     got = out.float().cpu().numpy().astype(np.float64)
     if rows is not None:
         got = got[rows]
@@ -226,7 +227,8 @@ def attn_case(mp, n, K, rows=None, dtype="bf16", r_c=8.5, seed=0):
     torch.cuda.synchronize()
     ctx.status_sync()
     model = oracle.Model.from_workload(wl, oracle_weights(w, dtype))
-    ref = oracle.attention(model, pos, nbr.cpu().numpy(), mask.cpu().numpy(), x_ref, rows=rows)
+    onbr, omask = oracle_padded(pos, wl.r_c, K, nbr, mask)
+    ref = oracle.attention(model, pos, onbr, omask, x_ref, rows=rows)
     got = out.float().cpu().numpy().astype(np.float64)
     return (got if rows is None else got[rows]), ref
 
@@ -293,8 +295,9 @@ def ef_case(mp, key, n=None, dtype=None, seed=0):
     torch.cuda.synchronize()
     ctx.status_sync()
     model = oracle.Model.from_workload(wl, oracle_weights(w, wl.dtype))
-    Eref, Fref, e_atom = oracle.energy_forces(model, pos, types, rp.cpu().numpy(),
-                                              ci.cpu().numpy(), gp, return_atom_energy=True)
+    orp, oci = oracle_csr(pos, wl.r_c, rp, ci, gp if G > 1 else None)
+    Eref, Fref, e_atom = oracle.energy_forces(model, pos, types, orp, oci, gp,
+                                              return_atom_energy=True)
     scale = np.array([np.abs(e_atom[gp[g]:gp[g + 1]]).sum() for g in range(G)])
     return E.cpu().numpy().astype(np.float64), F.cpu().numpy().astype(np.float64), Eref, Fref, scale
 

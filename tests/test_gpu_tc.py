@@ -12,7 +12,7 @@ import torch
 
 import oracle
 from atomistic_neighbor_list_b200 import synth
-from helpers import TOL_BF16_FEAT, features_for, normwise, oracle_weights
+from helpers import TOL_BF16_FEAT, features_for, normwise, oracle_csr, oracle_weights
 
 pytestmark = pytest.mark.gpu
 
@@ -40,9 +40,10 @@ def run_case(mp, pos, r_c=5.0, n_rbf=50, block=0, seed=0):
     torch.cuda.synchronize()
     ctx.status_sync()
     model = oracle.Model.from_workload(wl, oracle_weights(w, "bf16"))
-    ref = oracle.cfconv(model, block, pos, rp.cpu().numpy(), ci.cpu().numpy(), x_ref)
+    orp, oci = oracle_csr(pos, r_c, rp, ci)
+    ref = oracle.cfconv(model, block, pos, orp, oci, x_ref)
     got = out.float().cpu().numpy()
-    return got, ref, rp.cpu().numpy()
+    return got, ref, orp
 
 
 def test_rows_longer_than_a_tile(mp):
@@ -125,8 +126,9 @@ def run_ef(mp, pos, r_c=5.0, n_rbf=50, seed=0):
     torch.cuda.synchronize()
     ctx.status_sync()
     model = oracle.Model.from_workload(wl, oracle_weights(w, "bf16"))
-    Eref, Fref, e_atom = oracle.energy_forces(model, pos, types, rp.cpu().numpy(),
-                                              ci.cpu().numpy(), return_atom_energy=True)
+    orp, oci = oracle_csr(pos, r_c, rp, ci)
+    Eref, Fref, e_atom = oracle.energy_forces(model, pos, types, orp, oci,
+                                              return_atom_energy=True)
     e_err = abs(float(E[0]) - Eref[0]) / np.abs(e_atom).sum()
     return e_err, rel_rms(F.cpu().numpy(), Fref), TOL_BF16_FORCE
 

@@ -401,3 +401,79 @@ def test_attention_logit_shift_invariance():
     model.w["p"] = model.w["p"] + 3.0
     o2 = oracle.attention(model, pos, nbr, mask, x)
     assert np.allclose(o1, o2, rtol=1e-12, atol=1e-13)
+
+
+# ----------------------------------------------------------------------------- molecular dynamics
+def test_verlet_free_flight_is_exact():
+    rng = np.random.default_rng(0)
+    r0, v0 = rng.normal(size=(5, 3)), rng.normal(size=(5, 3))
+    zero = lambda r: (np.zeros(1), np.zeros_like(r))  # noqa: E731
+    r, v, f, e = oracle.velocity_verlet(zero, r0, v0, np.zeros((5, 3)), 0.1, 7)
+    assert np.allclose(r, r0 + 0.7 * v0, rtol=0, atol=1e-12) and np.array_equal(v, v0)
+
+
+def test_verlet_harmonic_closed_form():
+    """F = -k x with per-atom masses. One velocity-Verlet step is the linear map
+    x' = c x + h v,  v' = -h w^2 s x + c v  (c = 1 - h^2 w^2 / 2, s = 1 - h^2 w^2 / 4, w^2 = k / m),
+    a rotation by theta = arccos(c) in the metric of the invariant v^2 + w^2 s x^2; so after n steps
+    x_n = x0 cos(n theta) + h v0 sin(n theta) / sin(theta), and v_n likewise."""
+    rng = np.random.default_rng(1)
+    k, h, n = 2.0, 0.05, 1000
+    im = np.array([1.0, 0.5, 2.0, 0.25])
+    x0, v0 = rng.normal(size=(4, 3)), rng.normal(size=(4, 3))
+    spring = lambda r: (np.array([0.5 * k * np.sum(r * r)]), -k * r)  # noqa: E731
+    x, v, _, _ = oracle.velocity_verlet(spring, x0, v0, -k * x0, h, n, inv_mass=im)
+    w2 = (k * im)[:, None]
+    c, s = 1 - h * h * w2 / 2, 1 - h * h * w2 / 4
+    th = np.arccos(c)
+    xn = x0 * np.cos(n * th) + h * v0 * np.sin(n * th) / np.sin(th)
+    vn = v0 * np.cos(n * th) - h * w2 * s * x0 * np.sin(n * th) / np.sin(th)
+    assert np.allclose(x, xn, rtol=0, atol=1e-9) and np.allclose(v, vn, rtol=0, atol=1e-9)
+    inv0 = v0 ** 2 + w2 * s * x0 ** 2
+    assert np.allclose(v ** 2 + w2 * s * x ** 2, inv0, rtol=1e-10, atol=0)
+
+
+def test_kinetic_energy_by_hand():
+    v = np.array([[1.0, 2.0, 2.0], [0.0, 3.0, 4.0], [1.0, 0.0, 0.0]])
+    im = np.array([0.5, 1.0, 0.25])
+    # m |v|^2 / 2: 2 * 9 / 2 = 9; 1 * 25 / 2 = 12.5; 4 * 1 / 2 = 2
+    assert np.allclose(oracle.kinetic_energy(v, im), [23.5])
+    assert np.allclose(oracle.kinetic_energy(v, im, graph_ptr=[0, 2, 3]), [21.5, 2.0])
+    assert np.allclose(oracle.kinetic_energy(v), [0.5 * (9 + 25 + 1)])
+
+
+@pytest.fixture(scope="module")
+def md_system(fd_system):
+    """The 64-atom system with a neighbor list built with a 1 A skin (kept for the whole run)."""
+    model, pos, types, _, _ = fd_system
+    rp, ci = oracle.neighbor_csr(pos, model.r_c + 1.0)
+    im = 1.0 / (1.0 + types.astype(np.float64))
+    v0 = np.random.default_rng(7).normal(size=(len(pos), 3)) * np.sqrt(im)[:, None] * 0.05
+    force = lambda r: oracle.energy_forces(model, r, types, rp, ci)  # noqa: E731
+    return force, pos.astype(np.float64), v0, im
+
+
+def test_verlet_schnet_time_reversible(md_system):
+    force, r0, v0, im = md_system
+    _, f0 = force(r0)
+    r, v, f, _ = oracle.velocity_verlet(force, r0, v0, f0, 0.02, 8, im)
+    assert np.abs(r - r0).max() > 1e-3
+    rb, vb, _, _ = oracle.velocity_verlet(force, r, -v, f, 0.02, 8, im)
+    assert np.abs(rb - r0).max() < 1e-10 and np.abs(vb + v0).max() < 1e-10
+
+
+def test_verlet_schnet_energy_error_second_order(md_system):
+    """Conservative forces: the total-energy error of the same trajectory shrinks 4x when dt
+    halves (the scheme is second order), and the neighbor list with skin stays valid."""
+    force, r0, v0, im = md_system
+    e0, f0 = force(r0)
+    etot0 = e0[0] + oracle.kinetic_energy(v0, im)[0]
+    err = []
+    for dt, n in ((0.02, 10), (0.01, 20)):
+        r, v, f, worst = r0, v0, f0, 0.0
+        for _ in range(n):
+            r, v, f, e = oracle.velocity_verlet(force, r, v, f, dt, 1, im)
+            worst = max(worst, abs(e[0] + oracle.kinetic_energy(v, im)[0] - etot0))
+        assert np.abs(r - r0).max() < 0.5  # below skin / 2
+        err.append(worst)
+    assert err[0] > 1e-6 and 3.6 < err[0] / err[1] < 4.4, err
