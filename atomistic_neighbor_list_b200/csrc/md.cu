@@ -1,0 +1,161 @@
+// Velocity-Verlet molecular dynamics with the model's forces (FlashSchNet page, s.3: MD steps of
+// replicated systems; Tessera page: the neighbor topology is reused across steps). One step:
+//   v += (dt/2) F/m;  r += dt v;  (E, F) = energy and forces at r;  v += (dt/2) F/m.
+// The whole step (2 small kernels around the energy/forces launches) is recorded once per call as
+// a CUDA graph and replayed n_steps times.
+#include <cmath>
+
+#include "mp_internal.cuh"
+
+namespace mp {
+namespace {
+
+// v += (dt/2) F im; r += dt v   (im: 1/m per atom, or null for unit masses)
+__global__ void k_kick_drift(int N, float* __restrict__ pos, float* __restrict__ vel,
+                             const float* __restrict__ forces, const float* __restrict__ im,
+                             float dt) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= N) return;
+  const float h = 0.5f * dt * (im ? im[i] : 1.f);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    const float v = fmaf(h, forces[3 * i + c], vel[3 * i + c]);
+    vel[3 * i + c] = v;
+    pos[3 * i + c] = fmaf(dt, v, pos[3 * i + c]);
+  }
+}
+
+// v += (dt/2) F im
+__global__ void k_kick(int N, float* __restrict__ vel, const float* __restrict__ forces,
+                       const float* __restrict__ im, float dt) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= N) return;
+  const float h = 0.5f * dt * (im ? im[i] : 1.f);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) vel[3 * i + c] = fmaf(h, forces[3 * i + c], vel[3 * i + c]);
+}
+
+// kinetic[g] = sum over the atoms of graph g of |v|^2 / (2 im), fixed-order reduction per graph
+__global__ void k_kinetic(int N, const int* __restrict__ graph_ptr, int n_graphs,
+                          const float* __restrict__ vel, const float* __restrict__ im,
+                          float* __restrict__ kinetic, int* status) {
+  __shared__ float s_part[256];
+  for (int g = blockIdx.x; g < n_graphs; g += gridDim.x) {
+    const int lo = graph_ptr ? graph_ptr[g] : 0, hi = graph_ptr ? graph_ptr[g + 1] : N;
+    if (lo < 0 || hi > N || hi < lo) {
+      if (threadIdx.x == 0) {
+        raise_status(status, kStatusBounds);
+        kinetic[g] = 0.f;
+      }
+      continue;
+    }
+    float s = 0.f;
+    for (int i = lo + threadIdx.x; i < hi; i += blockDim.x) {
+      const float vx = vel[3 * i], vy = vel[3 * i + 1], vz = vel[3 * i + 2];
+      s += 0.5f * (vx * vx + vy * vy + vz * vz) / (im ? im[i] : 1.f);
+    }
+    s_part[threadIdx.x] = s;
+    __syncthreads();
+    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+      if (threadIdx.x < w) s_part[threadIdx.x] += s_part[threadIdx.x + w];
+      __syncthreads();
+    }
+    if (threadIdx.x == 0) kinetic[g] = s_part[0];
+    __syncthreads();
+  }
+}
+
+}  // namespace
+
+int md_step_launches(mp_ctx* c, int N, long long E, float* pos, float* vel, float* forces,
+                     const float* inv_mass, float dt, const int* types, const int* row_ptr,
+                     const int* col_idx, const int* graph_ptr, int n_graphs, float* energy,
+                     cudaStream_t s) {
+  const int blocks = (N + 255) / 256;
+  int rc = launch(c, K_MD, k_kick_drift, dim3(blocks), dim3(256), 0, s, N, pos, vel,
+                  (const float*)forces, inv_mass, dt);
+  if (rc == MP_OK)
+    rc = energy_forces_launches(c, N, E, pos, types, row_ptr, col_idx, graph_ptr, n_graphs,
+                                energy, forces, s);
+  if (rc == MP_OK)
+    rc = launch(c, K_MD, k_kick, dim3(blocks), dim3(256), 0, s, N, vel, (const float*)forces,
+                inv_mass, dt);
+  return rc;
+}
+
+int md_kinetic(mp_ctx* c, int N, const int* graph_ptr, int n_graphs, const float* vel,
+               const float* inv_mass, float* kinetic, cudaStream_t s) {
+  const int grid = n_graphs < 4 * c->num_sms ? n_graphs : 4 * c->num_sms;
+  return launch(c, K_MD, k_kinetic, dim3(grid), dim3(256), 0, s, N, graph_ptr, n_graphs, vel,
+                inv_mass, kinetic, c->status_d);
+}
+
+}  // namespace mp
+
+extern "C" int mp_md_verlet(mp_ctx* c, int N, long long E, float* pos, float* vel, float* forces,
+                            const float* inv_mass, float dt, int n_steps, const int* types,
+                            const int* row_ptr, const int* col_idx, const int* graph_ptr,
+                            int n_graphs, float* energy, float* kinetic, void* stream) {
+  using namespace mp;
+  if (!c || N < 0 || E < 0 || n_steps < 0 || !row_ptr || !energy || n_graphs < 1 ||
+      (N > 0 && (!pos || !vel || !forces || !types)) || (E > 0 && !col_idx) ||
+      (!graph_ptr && n_graphs != 1) || !std::isfinite(dt))
+    return MP_ERR_INVALID_ARG;
+  if (N > c->cfg.max_atoms || E > c->cfg.max_edges || n_graphs > c->cfg.max_graphs)
+    return MP_ERR_CAPACITY;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (c->cfg.validate) {
+    const int rc = launch_validate_csr(c, N, E, row_ptr, col_idx, graph_ptr, n_graphs, true, s);
+    if (rc != MP_OK) return rc;
+  }
+  if (N == 0 || n_steps == 0) {  // no atoms: energies are zero; no steps: kinetic only
+    int rc = MP_OK;
+    if (N == 0 && n_steps > 0)
+      rc = energy_forces_launches(c, 0, E, pos, types, row_ptr, col_idx, graph_ptr, n_graphs,
+                                  energy, forces, s);
+    if (rc == MP_OK && kinetic)
+      rc = md_kinetic(c, N, graph_ptr, n_graphs, vel, inv_mass, kinetic, s);
+    return rc;
+  }
+  // record one step as a graph and replay it, where the stream allows (as mp_energy_forces)
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  const bool use_graph = c->graphs && !c->graphs_broken && !c->profiling && s != nullptr &&
+                         cudaStreamIsCapturing(s, &cap) == cudaSuccess &&
+                         cap == cudaStreamCaptureStatusNone;
+  int rc = MP_OK;
+  cudaGraphExec_t ex = nullptr;
+  long long per_step = 0;
+  if (use_graph) {
+    const long long l0 = c->launches;
+    cudaGraph_t g = nullptr;
+    rc = cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal) == cudaSuccess ? MP_OK
+                                                                                  : MP_ERR_CUDA;
+    if (rc == MP_OK) {
+      rc = md_step_launches(c, N, E, pos, vel, forces, inv_mass, dt, types, row_ptr, col_idx,
+                            graph_ptr, n_graphs, energy, s);
+      if (cudaStreamEndCapture(s, &g) != cudaSuccess && rc == MP_OK) rc = MP_ERR_CUDA;
+    }
+    if (rc == MP_OK && (!g || cudaGraphInstantiate(&ex, g, 0) != cudaSuccess)) rc = MP_ERR_CUDA;
+    if (g) cudaGraphDestroy(g);
+    per_step = c->launches - l0;
+    c->launches = l0;
+    if (rc != MP_OK) {
+      cudaGetLastError();
+      c->graphs_broken = true;
+      ex = nullptr;
+      rc = MP_OK;
+    }
+  }
+  for (int st = 0; st < n_steps && rc == MP_OK; ++st) {
+    if (ex) {
+      rc = cudaGraphLaunch(ex, s) == cudaSuccess ? MP_OK : MP_ERR_CUDA;
+      c->launches += per_step;
+    } else {
+      rc = md_step_launches(c, N, E, pos, vel, forces, inv_mass, dt, types, row_ptr, col_idx,
+                            graph_ptr, n_graphs, energy, s);
+    }
+  }
+  if (ex) cudaGraphExecDestroy(ex);  // safe while a launch is pending: it completes first
+  if (rc == MP_OK && kinetic) rc = md_kinetic(c, N, graph_ptr, n_graphs, vel, inv_mass, kinetic, s);
+  return rc;
+}

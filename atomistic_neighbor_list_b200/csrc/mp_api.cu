@@ -14,7 +14,7 @@ const char* kernel_name(int id) {
   static const char* names[K_NUM] = {
       "embed", "dense", "readout_energy", "readout_bwd", "graph_energy_sum", "cfconv_fwd_simt",
       "cfconv_bwd_simt", "attn_simt", "validate_csr", "cfconv_fwd_tc", "cfconv_bwd_tc",
-      "attn_tc", "dense_tc"};
+      "attn_tc", "dense_tc", "md_integrate"};
   return (id >= 0 && id < K_NUM) ? names[id] : "?";
 }
 
@@ -304,7 +304,7 @@ extern "C" int mp_attn_fwd(mp_ctx* c, int N, int K, const float* pos, const int*
 }
 
 // The launches of one energy + forces evaluation (arguments already checked).
-static int energy_forces_launches(mp_ctx* c, int N, long long E, const float* pos, const int* types,
+int mp::energy_forces_launches(mp_ctx* c, int N, long long E, const float* pos, const int* types,
                                   const int* row_ptr, const int* col_idx, const int* graph_ptr,
                                   int n_graphs, float* energy, float* forces, cudaStream_t s) {
   const int F = c->cfg.F, Fh = F / 2, B = c->cfg.n_blocks;

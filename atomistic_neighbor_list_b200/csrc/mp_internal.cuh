@@ -34,7 +34,7 @@ struct FilterW {
 enum KernelId : int {
   K_EMBED = 0, K_DENSE, K_READOUT_E, K_READOUT_BWD, K_GRAPH_SUM, K_CFCONV_FWD_SIMT,
   K_CFCONV_BWD_SIMT, K_ATTN_SIMT, K_VALIDATE, K_CFCONV_FWD_TC, K_CFCONV_BWD_TC, K_ATTN_TC,
-  K_DENSE_TC, K_NUM
+  K_DENSE_TC, K_MD, K_NUM
 };
 const char* kernel_name(int id);
 
@@ -175,6 +175,10 @@ int launch_attn_simt(mp_ctx*, int N, int K, const float* pos, const int* nbr,
                      const unsigned char* mask, const void* x, void* out, cudaStream_t);
 int launch_validate_csr(mp_ctx*, int N, long long E, const int* row_ptr, const int* col_idx,
                         const int* graph_ptr, int n_graphs, bool need_sym, cudaStream_t);
+// The kernel sequence of one energy + forces evaluation (mp_api.cu), without validation or graphs.
+int energy_forces_launches(mp_ctx*, int N, long long E, const float* pos, const int* types,
+                           const int* row_ptr, const int* col_idx, const int* graph_ptr,
+                           int n_graphs, float* energy, float* forces, cudaStream_t);
 
 FilterW filter_of(const mp_ctx* ctx, int block);
 Radial radial_of(const mp_ctx* ctx);

@@ -66,6 +66,8 @@ def _load():
         "mp_profile_get": (i32, [vp, i32, POINTER(c_char_p), POINTER(c_double), POINTER(i64)]),
         "mp_launch_count": (i64, [vp]),
         "mp_set_graphs": (i32, [vp, i32]),
+        "mp_md_verlet": (i32, [vp, i32, i64, vp, vp, vp, vp, c_float, i32, vp, vp, vp, vp, i32,
+                               vp, vp, vp]),
         "mp_selftest_tc": (i32, [POINTER(i32)]),
         "mp_attn_fwd_noalloc": (i32, [POINTER(MpConfig), POINTER(MpWeights), i32, i32, vp, vp, vp,
                                       vp, vp, vp, vp]),
@@ -82,7 +84,8 @@ lib = _load()
 EXPORTED = ("mp_init", "mp_destroy", "mp_strerror", "mp_status_sync", "mp_neighbor_csr",
             "mp_neighbor_padded", "mp_cfconv_fwd", "mp_attn_fwd", "mp_energy_forces",
             "mp_profile_begin", "mp_profile_end", "mp_profile_get", "mp_launch_count",
-            "mp_attn_fwd_noalloc", "mp_selftest_tc", "mp_set_graphs")
+            "mp_attn_fwd_noalloc", "mp_selftest_tc", "mp_set_graphs",
+            "mp_md_verlet")
 NOALLOC_MAX_NF = 524288  # MP_NOALLOC_MAX_NF: largest N * F mp_attn_fwd_noalloc accepts
 
 
@@ -233,6 +236,37 @@ class Context:
 
     def launch_count(self) -> int:
         return int(lib.mp_launch_count(self._ctx))
+
+    def md_verlet(self, pos, vel, forces, types, row_ptr, col_idx, n_steps, dt, inv_mass=None,
+                  graph_ptr=None, energy=None, kinetic=None, stream=None):
+        """mp_md_verlet: n_steps velocity-Verlet steps in place on pos, vel, forces (forces must
+        hold the forces at pos on entry). The CSR is kept: build it with a skin. Returns
+        (energy, kinetic) of the last step; kinetic is computed when passed or requested as True."""
+        N = pos.shape[0]
+        _need(pos, "pos", torch.float32, (N, 3))
+        _need(vel, "vel", torch.float32, (N, 3))
+        _need(forces, "forces", torch.float32, (N, 3))
+        _need(types, "types", torch.int32, (N,))
+        _need(row_ptr, "row_ptr", torch.int32, (N + 1,))
+        _need(col_idx, "col_idx", torch.int32)
+        if inv_mass is not None:
+            _need(inv_mass, "inv_mass", torch.float32, (N,))
+        G = 1
+        if graph_ptr is not None:
+            _need(graph_ptr, "graph_ptr", torch.int32)
+            G = graph_ptr.numel() - 1
+        if energy is None:
+            energy = torch.empty(G, dtype=torch.float32, device=pos.device)
+        if kinetic is True:
+            kinetic = torch.empty(G, dtype=torch.float32, device=pos.device)
+        _need(energy, "energy", torch.float32, (G,))
+        if kinetic is not None:
+            _need(kinetic, "kinetic", torch.float32, (G,))
+        _check(lib.mp_md_verlet(self._ctx, N, col_idx.numel(), _ptr(pos), _ptr(vel), _ptr(forces),
+                                _ptr(inv_mass), float(dt), int(n_steps), _ptr(types),
+                                _ptr(row_ptr), _ptr(col_idx), _ptr(graph_ptr), G, _ptr(energy),
+                                _ptr(kinetic), _stream(stream)), "mp_md_verlet")
+        return energy, kinetic
 
     def set_graphs(self, on: bool):
         """Record / replay energy_forces as a CUDA graph (default on; see mp_set_graphs)."""

@@ -207,6 +207,31 @@ int mp_energy_forces(mp_ctx* ctx, int N, long long E, const float* pos, const in
  * the recorded graph. Errors: MP_ERR_INVALID_ARG.                                            */
 int mp_set_graphs(mp_ctx* ctx, int on);
 
+/* n_steps of velocity-Verlet molecular dynamics driven by mp_energy_forces [TS: the MD engine
+ * integrates the atoms locally each step and keeps the neighbor topology while coordinates move;
+ * CUDA graphs replay the fixed-shape step. FS: MD of batched replicas, throughput in
+ * timestep x molecule per second]. One step, for every atom i:
+ *   v_i += (dt/2) F_i / m_i;  r_i += dt v_i;  (energy, F) = mp_energy_forces(r);
+ *   v_i += (dt/2) F_i / m_i.
+ *   pos, vel, forces: float32 [N][3] (device), updated in place. On entry `forces` must hold the
+ *     forces at `pos` (from mp_energy_forces, or a previous call); on return pos, vel, forces and
+ *     energy belong to the last step.
+ *   inv_mass: float32 [N] 1/m_i (device), or NULL for unit masses. dt: time step (any finite value;
+ *     units are the caller's, consistent with the energy unit and masses).
+ *   The CSR (row_ptr, col_idx, graph_ptr) is NOT rebuilt: it must stay a superset of the pairs
+ *     within r_c for all n_steps, e.g. built with cutoff r_c + skin and rebuilt by the caller
+ *     before any atom has moved skin / 2 (pairs beyond r_c contribute exactly 0).
+ *   kinetic: float32 [n_graphs] (device), or NULL: per-graph kinetic energy sum m_i |v_i|^2 / 2
+ *     after the last step (fixed-order reduction).
+ *   On a non-default stream with graphs on, the step is recorded once as a CUDA graph and
+ *   replayed n_steps times; otherwise its kernels are launched step by step. n_steps = 0 only
+ *   computes kinetic. Errors: MP_ERR_INVALID_ARG (also for a non-finite dt), MP_ERR_CAPACITY,
+ *   MP_ERR_CUDA, CSR errors (validate, checked once per call).                              */
+int mp_md_verlet(mp_ctx* ctx, int N, long long E, float* pos, float* vel, float* forces,
+                 const float* inv_mass, float dt, int n_steps, const int* types,
+                 const int* row_ptr, const int* col_idx, const int* graph_ptr, int n_graphs,
+                 float* energy, float* kinetic, void* stream);
+
 /* Kernel timing for measurement. mp_profile_begin makes later calls record a CUDA event pair
  * around every kernel they launch (on the caller's stream); mp_profile_end synchronises the
  * stream and folds the pairs into per-kernel totals, readable by index with mp_profile_get
