@@ -65,6 +65,16 @@ __global__ void k_kinetic(int N, const int* __restrict__ graph_ptr, int n_graphs
   }
 }
 
+// flag = 1 when some atom has moved more than sqrt(lim2) from its reference position
+__global__ void k_displaced(int N, const float* __restrict__ pos, const float* __restrict__ ref,
+                            float lim2, int* __restrict__ flag) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= N) return;
+  const float dx = pos[3 * i] - ref[3 * i], dy = pos[3 * i + 1] - ref[3 * i + 1],
+              dz = pos[3 * i + 2] - ref[3 * i + 2];
+  if (dx * dx + dy * dy + dz * dz > lim2) *flag = 1;
+}
+
 }  // namespace
 
 int md_step_launches(mp_ctx* c, int N, long long E, float* pos, float* vel, float* forces,
@@ -88,6 +98,67 @@ int md_kinetic(mp_ctx* c, int N, const int* graph_ptr, int n_graphs, const float
   const int grid = n_graphs < 4 * c->num_sms ? n_graphs : 4 * c->num_sms;
   return launch(c, K_MD, k_kinetic, dim3(grid), dim3(256), 0, s, N, graph_ptr, n_graphs, vel,
                 inv_mass, kinetic, c->status_d);
+}
+
+// One recorded step, replayed: capture succeeds on a non-default stream that is not already
+// capturing; otherwise ex stays null and the caller launches the step's kernels itself.
+struct StepGraph {
+  cudaGraphExec_t ex = nullptr;
+  long long per_step = 0;
+  ~StepGraph() { reset(); }
+  void reset() {
+    if (ex) cudaGraphExecDestroy(ex);  // a pending launch completes first
+    ex = nullptr;
+  }
+};
+
+bool can_record(mp_ctx* c, cudaStream_t s) {
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  return c->graphs && !c->graphs_broken && !c->profiling && s != nullptr &&
+         cudaStreamIsCapturing(s, &cap) == cudaSuccess && cap == cudaStreamCaptureStatusNone;
+}
+
+void record_step(mp_ctx* c, StepGraph& sg, int N, long long E, float* pos, float* vel,
+                 float* forces, const float* inv_mass, float dt, const int* types,
+                 const int* row_ptr, const int* col_idx, const int* graph_ptr, int n_graphs,
+                 float* energy, cudaStream_t s) {
+  sg.reset();
+  if (!can_record(c, s)) return;
+  const long long l0 = c->launches;
+  cudaGraph_t g = nullptr;
+  int rc = cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal) == cudaSuccess ? MP_OK
+                                                                                    : MP_ERR_CUDA;
+  if (rc == MP_OK) {
+    rc = md_step_launches(c, N, E, pos, vel, forces, inv_mass, dt, types, row_ptr, col_idx,
+                          graph_ptr, n_graphs, energy, s);
+    if (cudaStreamEndCapture(s, &g) != cudaSuccess && rc == MP_OK) rc = MP_ERR_CUDA;
+  }
+  if (rc == MP_OK && (!g || cudaGraphInstantiate(&sg.ex, g, 0) != cudaSuccess)) rc = MP_ERR_CUDA;
+  if (g) cudaGraphDestroy(g);
+  sg.per_step = c->launches - l0;
+  c->launches = l0;
+  if (rc != MP_OK) {  // plain launches from now on for this context
+    cudaGetLastError();
+    c->graphs_broken = true;
+    sg.ex = nullptr;
+  }
+}
+
+int run_steps(mp_ctx* c, StepGraph& sg, int n, int N, long long E, float* pos, float* vel,
+              float* forces, const float* inv_mass, float dt, const int* types, const int* row_ptr,
+              const int* col_idx, const int* graph_ptr, int n_graphs, float* energy,
+              cudaStream_t s) {
+  int rc = MP_OK;
+  for (int st = 0; st < n && rc == MP_OK; ++st) {
+    if (sg.ex) {
+      rc = cudaGraphLaunch(sg.ex, s) == cudaSuccess ? MP_OK : MP_ERR_CUDA;
+      c->launches += sg.per_step;
+    } else {
+      rc = md_step_launches(c, N, E, pos, vel, forces, inv_mass, dt, types, row_ptr, col_idx,
+                            graph_ptr, n_graphs, energy, s);
+    }
+  }
+  return rc;
 }
 
 }  // namespace mp
@@ -117,45 +188,82 @@ extern "C" int mp_md_verlet(mp_ctx* c, int N, long long E, float* pos, float* ve
       rc = md_kinetic(c, N, graph_ptr, n_graphs, vel, inv_mass, kinetic, s);
     return rc;
   }
-  // record one step as a graph and replay it, where the stream allows (as mp_energy_forces)
-  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-  const bool use_graph = c->graphs && !c->graphs_broken && !c->profiling && s != nullptr &&
-                         cudaStreamIsCapturing(s, &cap) == cudaSuccess &&
-                         cap == cudaStreamCaptureStatusNone;
-  int rc = MP_OK;
-  cudaGraphExec_t ex = nullptr;
-  long long per_step = 0;
-  if (use_graph) {
-    const long long l0 = c->launches;
-    cudaGraph_t g = nullptr;
-    rc = cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal) == cudaSuccess ? MP_OK
-                                                                                  : MP_ERR_CUDA;
-    if (rc == MP_OK) {
-      rc = md_step_launches(c, N, E, pos, vel, forces, inv_mass, dt, types, row_ptr, col_idx,
-                            graph_ptr, n_graphs, energy, s);
-      if (cudaStreamEndCapture(s, &g) != cudaSuccess && rc == MP_OK) rc = MP_ERR_CUDA;
+  StepGraph sg;
+  record_step(c, sg, N, E, pos, vel, forces, inv_mass, dt, types, row_ptr, col_idx, graph_ptr,
+              n_graphs, energy, s);
+  int rc = run_steps(c, sg, n_steps, N, E, pos, vel, forces, inv_mass, dt, types, row_ptr,
+                     col_idx, graph_ptr, n_graphs, energy, s);
+  if (rc == MP_OK && kinetic) rc = md_kinetic(c, N, graph_ptr, n_graphs, vel, inv_mass, kinetic, s);
+  return rc;
+}
+
+extern "C" int mp_md_run(mp_ctx* c, int N, float* pos, float* vel, float* forces,
+                         const float* inv_mass, float dt, int n_steps, const int* types,
+                         const int* graph_ptr, int n_graphs, float skin, int rebuild_every,
+                         float max_disp, int check_every, int* row_ptr, int* col_idx,
+                         long long capacity, long long* n_edges, float* energy, float* kinetic,
+                         int* n_builds, void* stream) {
+  using namespace mp;
+  if (!c || N < 0 || n_steps < 0 || !row_ptr || !energy || n_graphs < 1 || !n_edges ||
+      (N > 0 && (!pos || !vel || !forces || !types)) || (capacity > 0 && !col_idx) ||
+      capacity < 0 || (!graph_ptr && n_graphs != 1) || !std::isfinite(dt) ||
+      !std::isfinite(skin) || skin < 0.f || !std::isfinite(max_disp) || rebuild_every < 0 ||
+      check_every < 1)
+    return MP_ERR_INVALID_ARG;
+  if (N > c->cfg.max_atoms || n_graphs > c->cfg.max_graphs) return MP_ERR_CAPACITY;
+  cudaStream_t s = (cudaStream_t)stream;
+  const float r_list = c->cfg.r_c + skin;
+  long long E = 0;
+  int builds = 0;
+  StepGraph sg;
+  // the list at the current positions, the reference positions, and energy/forces with it
+  auto build = [&]() -> int {
+    int rc = mp_neighbor_csr(N, pos, graph_ptr, n_graphs, r_list, row_ptr, col_idx, capacity, &E,
+                             stream);
+    *n_edges = E;
+    if (rc != MP_OK) return rc;
+    if (E > c->cfg.max_edges) return MP_ERR_CAPACITY;
+    ++builds;
+    if (N > 0 && cudaMemcpyAsync(c->md_ref, pos, sizeof(float) * 3 * (size_t)N,
+                                 cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return MP_ERR_CUDA;
+    rc = energy_forces_launches(c, N, E, pos, types, row_ptr, col_idx, graph_ptr, n_graphs,
+                                energy, forces, s);
+    if (rc == MP_OK && N > 0)
+      record_step(c, sg, N, E, pos, vel, forces, inv_mass, dt, types, row_ptr, col_idx,
+                  graph_ptr, n_graphs, energy, s);
+    return rc;
+  };
+  int rc = build();
+  const float lim2 = max_disp * max_disp;
+  int done = 0, since = 0;
+  while (rc == MP_OK && N > 0 && done < n_steps) {
+    int chunk = n_steps - done < check_every ? n_steps - done : check_every;
+    if (rebuild_every > 0 && rebuild_every - since < chunk) chunk = rebuild_every - since;
+    rc = run_steps(c, sg, chunk, N, E, pos, vel, forces, inv_mass, dt, types, row_ptr, col_idx,
+                   graph_ptr, n_graphs, energy, s);
+    done += chunk;
+    since += chunk;
+    if (rc != MP_OK || done == n_steps) break;
+    bool rebuild = rebuild_every > 0 && since >= rebuild_every;
+    if (!rebuild && max_disp > 0.f) {  // early rebuild: one flag read per check
+      cudaMemsetAsync(c->md_flag, 0, sizeof(int), s);
+      rc = launch(c, K_MD, k_displaced, dim3((N + 255) / 256), dim3(256), 0, s, N,
+                  (const float*)pos, (const float*)c->md_ref, lim2, c->md_flag);
+      if (rc != MP_OK) break;
+      cudaMemcpyAsync(c->md_flag_h, c->md_flag, sizeof(int), cudaMemcpyDeviceToHost, s);
+      if (cudaStreamSynchronize(s) != cudaSuccess) {
+        rc = MP_ERR_CUDA;
+        break;
+      }
+      rebuild = *c->md_flag_h != 0;
     }
-    if (rc == MP_OK && (!g || cudaGraphInstantiate(&ex, g, 0) != cudaSuccess)) rc = MP_ERR_CUDA;
-    if (g) cudaGraphDestroy(g);
-    per_step = c->launches - l0;
-    c->launches = l0;
-    if (rc != MP_OK) {
-      cudaGetLastError();
-      c->graphs_broken = true;
-      ex = nullptr;
-      rc = MP_OK;
+    if (rebuild) {
+      rc = build();
+      since = 0;
     }
   }
-  for (int st = 0; st < n_steps && rc == MP_OK; ++st) {
-    if (ex) {
-      rc = cudaGraphLaunch(ex, s) == cudaSuccess ? MP_OK : MP_ERR_CUDA;
-      c->launches += per_step;
-    } else {
-      rc = md_step_launches(c, N, E, pos, vel, forces, inv_mass, dt, types, row_ptr, col_idx,
-                            graph_ptr, n_graphs, energy, s);
-    }
-  }
-  if (ex) cudaGraphExecDestroy(ex);  // safe while a launch is pending: it completes first
+  if (n_builds) *n_builds = builds;
   if (rc == MP_OK && kinetic) rc = md_kinetic(c, N, graph_ptr, n_graphs, vel, inv_mass, kinetic, s);
   return rc;
 }

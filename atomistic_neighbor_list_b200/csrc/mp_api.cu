@@ -209,7 +209,8 @@ extern "C" int mp_init(mp_ctx** out_ctx, const mp_config* cfg, const mp_weights*
                     nf * 4,            // g_x
                     nf * st,           // g_m
                     nf * 4,            // grad_h
-                    nf * 4, nf * 4};   // q, k
+                    nf * 4, nf * 4,    // q, k
+                    N * 3 * 4};        // md_ref
   size_t ws = 0;
   for (size_t v : sizes) ws += align_up(v, 256);
   char* wsb = nullptr;
@@ -235,12 +236,15 @@ extern "C" int mp_init(mp_ctx** out_ctx, const mp_config* cfg, const mp_weights*
   c->grad_h = (float*)take(sizes[8]);
   c->q = (float*)take(sizes[9]);
   c->k = (float*)take(sizes[10]);
-  if (cudaMalloc(&c->status_d, sizeof(int)) != cudaSuccess ||
-      cudaMallocHost(&c->status_h, sizeof(int)) != cudaSuccess) {
+  c->md_ref = (float*)take(sizes[11]);
+  if (cudaMalloc(&c->status_d, 4 * sizeof(int)) != cudaSuccess ||
+      cudaMallocHost(&c->status_h, 4 * sizeof(int)) != cudaSuccess) {
     free_ctx(c);
     return MP_ERR_CUDA;
   }
-  cudaMemsetAsync(c->status_d, 0, sizeof(int), s);
+  c->md_flag = c->status_d + 1;
+  c->md_flag_h = c->status_h + 1;
+  cudaMemsetAsync(c->status_d, 0, 4 * sizeof(int), s);
   int rc = tc_prepare(c, s);  // packed operand images for the tensor-core kernels
   if (rc != MP_OK || cudaStreamSynchronize(s) != cudaSuccess) {
     free_ctx(c);

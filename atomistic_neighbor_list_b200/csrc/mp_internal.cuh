@@ -70,8 +70,11 @@ struct mp_ctx {
   float* grad_h = nullptr;                // [N][F] dE/dh
   float* q = nullptr;                     // [N][F] attention queries
   float* k = nullptr;                     // [N][F] attention keys
-  int* status_d = nullptr;                // device status bits
+  float* md_ref = nullptr;                // [N][3] positions at the last neighbor-list build
+  int* status_d = nullptr;                // device status bits (then the MD displacement flag)
   int* status_h = nullptr;                // pinned host copy
+  int* md_flag = nullptr;                 // status_d + 1: an atom moved past the rebuild limit
+  int* md_flag_h = nullptr;               // status_h + 1
   long long launches = 0;
   // CUDA graph of the last energy/forces call, replayed when a call repeats its arguments
   bool graphs = true, graphs_broken = false;

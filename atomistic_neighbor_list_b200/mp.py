@@ -68,6 +68,8 @@ def _load():
         "mp_set_graphs": (i32, [vp, i32]),
         "mp_md_verlet": (i32, [vp, i32, i64, vp, vp, vp, vp, c_float, i32, vp, vp, vp, vp, i32,
                                vp, vp, vp]),
+        "mp_md_run": (i32, [vp, i32, vp, vp, vp, vp, c_float, i32, vp, vp, i32, c_float, i32,
+                            c_float, i32, vp, vp, i64, POINTER(i64), vp, vp, POINTER(i32), vp]),
         "mp_selftest_tc": (i32, [POINTER(i32)]),
         "mp_attn_fwd_noalloc": (i32, [POINTER(MpConfig), POINTER(MpWeights), i32, i32, vp, vp, vp,
                                       vp, vp, vp, vp]),
@@ -85,7 +87,7 @@ EXPORTED = ("mp_init", "mp_destroy", "mp_strerror", "mp_status_sync", "mp_neighb
             "mp_neighbor_padded", "mp_cfconv_fwd", "mp_attn_fwd", "mp_energy_forces",
             "mp_profile_begin", "mp_profile_end", "mp_profile_get", "mp_launch_count",
             "mp_attn_fwd_noalloc", "mp_selftest_tc", "mp_set_graphs",
-            "mp_md_verlet")
+            "mp_md_verlet", "mp_md_run")
 NOALLOC_MAX_NF = 524288  # MP_NOALLOC_MAX_NF: largest N * F mp_attn_fwd_noalloc accepts
 
 
@@ -267,6 +269,51 @@ class Context:
                                 _ptr(row_ptr), _ptr(col_idx), _ptr(graph_ptr), G, _ptr(energy),
                                 _ptr(kinetic), _stream(stream)), "mp_md_verlet")
         return energy, kinetic
+
+    def md_run(self, pos, vel, types, n_steps, dt, skin, capacity, rebuild_every=0,
+               max_disp=None, check_every=1, inv_mass=None, graph_ptr=None, forces=None,
+               energy=None, kinetic=None, row_ptr=None, col_idx=None, stream=None):
+        """mp_md_run: n_steps velocity-Verlet steps that build and maintain their own neighbor
+        list (cutoff r_c + skin; rebuilt every rebuild_every steps and whenever an atom moved more
+        than max_disp, default skin / 2, since the last build). Returns a dict with energy,
+        kinetic (when passed or True), forces, row_ptr, col_idx (the last list, E entries),
+        n_edges and n_builds."""
+        N = pos.shape[0]
+        _need(pos, "pos", torch.float32, (N, 3))
+        _need(vel, "vel", torch.float32, (N, 3))
+        _need(types, "types", torch.int32, (N,))
+        if inv_mass is not None:
+            _need(inv_mass, "inv_mass", torch.float32, (N,))
+        G = 1
+        if graph_ptr is not None:
+            _need(graph_ptr, "graph_ptr", torch.int32)
+            G = graph_ptr.numel() - 1
+        dev = pos.device
+        forces = torch.empty((N, 3), dtype=torch.float32, device=dev) if forces is None else forces
+        energy = torch.empty(G, dtype=torch.float32, device=dev) if energy is None else energy
+        if kinetic is True:
+            kinetic = torch.empty(G, dtype=torch.float32, device=dev)
+        row_ptr = torch.empty(N + 1, dtype=torch.int32, device=dev) if row_ptr is None else row_ptr
+        if col_idx is None:
+            col_idx = torch.empty(max(int(capacity), 1), dtype=torch.int32, device=dev)
+        _need(forces, "forces", torch.float32, (N, 3))
+        _need(energy, "energy", torch.float32, (G,))
+        if kinetic is not None:
+            _need(kinetic, "kinetic", torch.float32, (G,))
+        _need(row_ptr, "row_ptr", torch.int32, (N + 1,))
+        _need(col_idx, "col_idx", torch.int32)
+        if col_idx.numel() < capacity:
+            raise ValueError("col_idx: fewer entries than capacity")
+        md = skin / 2 if max_disp is None else max_disp
+        n_edges, n_builds = c_longlong(0), c_int(0)
+        _check(lib.mp_md_run(self._ctx, N, _ptr(pos), _ptr(vel), _ptr(forces), _ptr(inv_mass),
+                             float(dt), int(n_steps), _ptr(types), _ptr(graph_ptr), G, float(skin),
+                             int(rebuild_every), float(md), int(check_every), _ptr(row_ptr),
+                             _ptr(col_idx), int(capacity), ctypes.byref(n_edges), _ptr(energy),
+                             _ptr(kinetic), ctypes.byref(n_builds), _stream(stream)), "mp_md_run")
+        return {"energy": energy, "kinetic": kinetic, "forces": forces, "row_ptr": row_ptr,
+                "col_idx": col_idx[: n_edges.value], "n_edges": n_edges.value,
+                "n_builds": n_builds.value}
 
     def set_graphs(self, on: bool):
         """Record / replay energy_forces as a CUDA graph (default on; see mp_set_graphs)."""

@@ -232,6 +232,31 @@ int mp_md_verlet(mp_ctx* ctx, int N, long long E, float* pos, float* vel, float*
                  const int* row_ptr, const int* col_idx, const int* graph_ptr, int n_graphs,
                  float* energy, float* kinetic, void* stream);
 
+/* Velocity-Verlet MD that maintains its own neighbor list [TS: the neighbor topology is reused
+ * while the coordinates move; it is rebuilt at a fixed step interval, or early, after a global
+ * check, once an atom has moved more than a displacement limit]. The call builds the list with
+ * cutoff r_c + skin at the current positions (mp_neighbor_csr into row_ptr / col_idx, capacity
+ * entries), evaluates energy and forces with it (`forces` need not hold anything on entry), then
+ * runs n_steps steps of mp_md_verlet's scheme. It rebuilds the list, and re-evaluates energy and
+ * forces at the current positions with the new list, after every rebuild_every steps (0: never
+ * on a schedule) and after any check that finds an atom more than max_disp from where it was at
+ * the last build (checked every check_every >= 1 steps; max_disp <= 0 disables it).
+ * The forces equal those of an exact r_c list at every step as long as no atom gets further than
+ * skin / 2 from its position at the last build between two checks; max_disp <= skin / 2 with
+ * check_every = 1 guarantees it.
+ *   row_ptr int32 [N+1], col_idx int32 [capacity] (device): the list, owned by the caller;
+ *   *n_edges (HOST) receives the edge count of the last build, *n_builds (HOST, or NULL) the
+ *   number of builds. Other arguments as mp_md_verlet. Each check and each build synchronises
+ *   `stream`; steps between checks are replayed from one recorded CUDA graph per build.
+ * Errors: MP_ERR_INVALID_ARG (non-finite dt, skin or max_disp, skin < 0, check_every < 1,
+ * rebuild_every < 0), MP_ERR_CAPACITY (a list larger than capacity or the context's max_edges:
+ * the call stops there, with pos / vel of the last completed step), MP_ERR_CUDA.             */
+int mp_md_run(mp_ctx* ctx, int N, float* pos, float* vel, float* forces, const float* inv_mass,
+              float dt, int n_steps, const int* types, const int* graph_ptr, int n_graphs,
+              float skin, int rebuild_every, float max_disp, int check_every, int* row_ptr,
+              int* col_idx, long long capacity, long long* n_edges, float* energy,
+              float* kinetic, int* n_builds, void* stream);
+
 /* Kernel timing for measurement. mp_profile_begin makes later calls record a CUDA event pair
  * around every kernel they launch (on the caller's stream); mp_profile_end synchronises the
  * stream and folds the pairs into per-kernel totals, readable by index with mp_profile_get

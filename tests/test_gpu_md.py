@@ -216,3 +216,72 @@ def test_md_no_atoms(mp):
     torch.cuda.synchronize()
     ctx.status_sync()
     assert torch.equal(e.cpu(), torch.zeros(2)) and torch.equal(k.cpu(), torch.zeros(2))
+
+
+# ----------------------------------------------------------------------------- list maintenance
+def fast_system(n=300, seed=5, vscale=1.5):
+    """fp32, one interaction block; velocities large enough that atoms cross the rebuild limit."""
+    wl = dataclasses.replace(synth.scaled(synth.WORKLOADS["cfg2"], n), dtype="fp32", n_blocks=1)
+    pos, _, types, im, _ = md_inputs(wl, seed)
+    v0 = (np.random.default_rng(seed + 20).normal(size=(n, 3)) * np.sqrt(im)[:, None] * vscale)
+    return wl, pos, types, im, v0.astype(np.float32)
+
+
+def test_md_run_matches_fresh_exact_lists(mp):
+    """mp_md_run keeps an r_c + skin list and rebuilds it when an atom has moved skin / 2; the
+    oracle's forces come from an exact r_c list built afresh at every evaluation. The two
+    trajectories agree, so no pair was ever missing from the kept list."""
+    wl, pos, types, im, v0 = fast_system()
+    skin, dt, steps = 0.5, 0.01, 40
+    cap = 2 * len(oracle.neighbor_csr(pos, wl.r_c + skin)[1]) + 1024
+    ctx = mp.Context.from_workload(wl, synth.make_weights(wl), max_atoms=len(pos), max_edges=cap)
+    p, v = dev(pos), dev(v0)
+    side = torch.cuda.Stream()  # a stream of its own: the steps are replayed from graphs
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        out = ctx.md_run(p, v, dev(types), steps, dt, skin, cap, inv_mass=dev(im), kinetic=True)
+    side.synchronize()
+    ctx.status_sync()
+    model = oracle.Model.from_workload(wl, synth.make_weights(wl))
+
+    def fresh(r):
+        rp, ci = oracle.neighbor_csr(r, wl.r_c)
+        return oracle.energy_forces(model, r, types, rp, ci)
+
+    e0, f0 = fresh(pos.astype(np.float64))
+    r, vr, fr, er = oracle.velocity_verlet(fresh, pos, v0, f0, dt, steps, im)
+    got = p.cpu().numpy().astype(np.float64)
+    assert np.abs(r - pos).max() > 2 * skin  # far enough that the list had to be rebuilt
+    assert out["n_builds"] >= 3
+    assert np.abs(got - r).max() <= 1e-3
+    assert rel_rms(v.cpu().numpy(), vr) <= 1e-3
+    assert rel_rms(out["forces"].cpu().numpy(), fr) <= 1e-3
+    # the list kept at the end holds every pair within r_c at the final positions
+    orp, oci = oracle.neighbor_csr(got.astype(np.float32), wl.r_c)
+    rp, ci = out["row_ptr"].cpu().numpy(), out["col_idx"].cpu().numpy()
+    kept = {(i, j) for i in range(len(got)) for j in ci[rp[i]:rp[i + 1]]}
+    need = {(i, j) for i in range(len(got)) for j in oci[orp[i]:orp[i + 1]]}
+    assert need <= kept
+
+
+def test_md_run_schedule_and_capacity(mp):
+    wl, pos, types, im, _ = fast_system(seed=6, vscale=0.0)
+    v0 = np.zeros_like(pos)
+    cap = 2 * len(oracle.neighbor_csr(pos, wl.r_c + 0.5)[1]) + 1024
+    ctx = mp.Context.from_workload(wl, synth.make_weights(wl), max_atoms=len(pos), max_edges=cap)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        out = ctx.md_run(dev(pos), dev(v0), dev(types), 25, 0.001, 0.5, cap, rebuild_every=10,
+                         max_disp=0.0)
+        assert out["n_builds"] == 3  # at the start, after 10 and after 20 steps
+        out = ctx.md_run(dev(pos), dev(v0), dev(types), 25, 0.001, 0.5, cap)
+        assert out["n_builds"] == 1  # atoms at rest never reach the displacement limit
+        with pytest.raises(mp.MpError) as err:
+            ctx.md_run(dev(pos), dev(v0), dev(types), 5, 0.001, 0.5, 10)
+        assert err.value.name == "MP_ERR_CAPACITY"
+        with pytest.raises(mp.MpError) as err:
+            ctx.md_run(dev(pos), dev(v0), dev(types), 5, 0.001, -0.5, cap)
+        assert err.value.name == "MP_ERR_INVALID_ARG"
+    side.synchronize()
+    ctx.status_sync()
