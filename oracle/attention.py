@@ -22,7 +22,7 @@ import math
 
 import numpy as np
 
-from .schnet import Model, filter_weights, gaussian_rbf
+from .schnet import Model, filter_weights, gaussian_rbf, gaussian_rbf_grad
 
 ROW_CHUNK = 256
 
@@ -61,3 +61,87 @@ def attention(model: Model, pos, nbr, mask, x, rows=None) -> np.ndarray:
         alpha = p / np.where(z > 0, z, 1.0)[:, None, :]
         out[c0:c0 + nc] = np.einsum("nkh,nkhd->nhd", alpha, v).reshape(nc, F)
     return out
+
+
+def attention_vjp(model: Model, pos, nbr, mask, x, g, rows=None):
+    """Gradients of L = sum_{i in rows} g_i . out_i with respect to x and the positions (float64).
+
+    Reverse-mode differentiation of ``attention`` (E2Former-V2 page, section 3.2: the backward of
+    the fused kernel; Tessera page: forces are gradients with respect to the positions). With
+    v_ij = x_j (.) W(d_ij), alpha the softmax over the valid slots of row i, per head h:
+
+        dalpha_ijh = sum_{c in h} g_i[c] v_ij[c]
+        dl_ijh     = alpha_ijh (dalpha_ijh - sum_j' alpha_ij'h dalpha_ij'h)
+        dL/dq_i    = sum_j dl_ijh k_jh / sqrt(D),      dL/dk_j += dl_ijh q_ih / sqrt(D)
+        dL/dx_j   += alpha_ijh g_i (.) W(d_ij)          (value path)
+        dL/dd_ij   = sum_c alpha g_i[c] x_j[c] W'(d_ij)[c] + sum_h dl_ijh sum_k e_k'(d_ij) P_kh
+        dL/dr_i   += dL/dd_ij (r_i - r_j) / d_ij,  dL/dr_j -= the same
+        dL/dx      = dL/dq Wq^T + dL/dk Wk^T + the value path.
+
+    A pair at d = 0 contributes no position gradient. Rows not in ``rows`` contribute nothing.
+    Returns (grad_x [N,F], grad_pos [N,3]).
+    """
+    w = model.w
+    H, D = model.n_heads, model.head_dim
+    pos64 = np.asarray(pos, dtype=np.float64)
+    x = np.asarray(x, dtype=np.float64)
+    g = np.asarray(g, dtype=np.float64)
+    nbr = np.asarray(nbr)
+    mask = np.asarray(mask)
+    n, K = nbr.shape
+    F = x.shape[1]
+    sel = np.arange(n) if rows is None else np.asarray(rows, dtype=np.int64)
+    sq = math.sqrt(D)
+    q = x @ w["Wq"]
+    kx = x @ w["Wk"]
+    gq = np.zeros((n, F))
+    gk = np.zeros((n, F))
+    gx = np.zeros((n, F))
+    gpos = np.zeros((n, 3))
+    for c0 in range(0, len(sel), ROW_CHUNK):
+        rws = sel[c0:c0 + ROW_CHUNK]
+        nc = len(rws)
+        valid = mask[rws] != 0
+        jj = np.where(valid, nbr[rws], 0).astype(np.int64)
+        vec = pos64[rws][:, None, :] - pos64[jj]
+        d = np.sqrt(np.sum(vec * vec, axis=2)).ravel()
+        e = gaussian_rbf(d, model.mu, model.gamma)
+        de = gaussian_rbf_grad(d, model.mu, model.gamma)
+        W, dW = filter_weights(model, 0, d, with_grad=True)
+        W = W.reshape(nc, K, F)
+        dW = dW.reshape(nc, K, F)
+        xj = x[jj]
+        v = (xj * W).reshape(nc, K, H, D)
+        qi = q[rws].reshape(nc, H, D)
+        kj = kx[jj].reshape(nc, K, H, D)
+        logits = (np.einsum("nhd,nkhd->nkh", qi, kj) / sq
+                  + (e @ w["P"]).reshape(nc, K, H) + w["p"][None, None, :])
+        logits = np.where(valid[:, :, None], logits, -np.inf)
+        has = valid.any(axis=1)
+        mx = np.where(has[:, None], np.max(np.where(has[:, None, None], logits, 0.0), axis=1), 0.0)
+        p = np.where(valid[:, :, None], np.exp(logits - mx[:, None, :]), 0.0)
+        z = p.sum(axis=1)
+        alpha = p / np.where(z > 0, z, 1.0)[:, None, :]
+        gi = g[rws].reshape(nc, H, D)
+        dalpha = np.einsum("nhd,nkhd->nkh", gi, v)
+        dl = alpha * (dalpha - np.sum(alpha * dalpha, axis=1)[:, None, :])
+        # logits: q_i and k_j
+        gq[rws] += (np.einsum("nkh,nkhd->nhd", dl, kj) / sq).reshape(nc, F)
+        dk = (dl[:, :, :, None] * qi[:, None, :, :] / sq).reshape(nc * K, F)
+        # value path
+        gv = (alpha[:, :, :, None] * gi[:, None, :, :]).reshape(nc, K, F)
+        dxj = (gv * W).reshape(nc * K, F)
+        keep = valid.ravel()
+        np.add.at(gk, jj.ravel()[keep], dk[keep])
+        np.add.at(gx, jj.ravel()[keep], dxj[keep])
+        # distance: the filter and the logit bias
+        s = (np.sum(gv * xj * dW, axis=2)
+             + np.einsum("nkh,nkh->nk", dl, (de @ w["P"]).reshape(nc, K, H))).ravel()
+        s = np.where(keep, s, 0.0)
+        safe = d > 0
+        u = np.where(safe[:, None], vec.reshape(nc * K, 3) / np.where(safe, d, 1.0)[:, None], 0.0)
+        su = s[:, None] * u
+        np.add.at(gpos, np.repeat(rws, K), su)
+        np.add.at(gpos, jj.ravel(), -su)
+    gx += gq @ w["Wq"].T + gk @ w["Wk"].T
+    return gx, gpos

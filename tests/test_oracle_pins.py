@@ -403,6 +403,76 @@ def test_attention_logit_shift_invariance():
     assert np.allclose(o1, o2, rtol=1e-12, atol=1e-13)
 
 
+@pytest.fixture(scope="module")
+def attn_system():
+    """24 atoms in a small box (up to 10 valid slots of 12 per row, some rows capped), F = 8."""
+    model, w, wl = small_model(F=8, R=6, n_heads=2, head_dim=4)
+    pos = (np.random.default_rng(21).uniform(0, 7.0, size=(24, 3))).astype(np.float64)
+    x = synth.node_features(24, 8, seed=5).astype(np.float64)
+    nbr, mask = oracle.neighbor_padded(pos.astype(np.float32), 5.0, 10)
+    g = np.random.default_rng(22).normal(size=(24, 8))
+    return model, pos, x, nbr, mask, g
+
+
+def _loss(model, pos, x, nbr, mask, g):
+    return float(np.sum(g * oracle.attention(model, pos, nbr, mask, x)))
+
+
+def test_attention_vjp_matches_central_differences(attn_system):
+    """The list is held fixed while an input moves by +-h (h = 1e-6): dL/dx and dL/dr against
+    central differences of L = sum g . out, every entry."""
+    model, pos, x, nbr, mask, g = attn_system
+    assert 0 < mask.sum(axis=1).min() and mask.sum(axis=1).max() == 10  # some rows are capped
+    gx, gpos = oracle.attention_vjp(model, pos, nbr, mask, x, g)
+    h = 1e-6
+    fdx = np.zeros_like(x)
+    for a in range(x.shape[0]):
+        for c in range(x.shape[1]):
+            xp, xm = x.copy(), x.copy()
+            xp[a, c] += h
+            xm[a, c] -= h
+            fdx[a, c] = (_loss(model, pos, xp, nbr, mask, g) - _loss(model, pos, xm, nbr, mask, g)) / (2 * h)
+    fdp = np.zeros_like(pos)
+    for a in range(pos.shape[0]):
+        for c in range(3):
+            pp, pm = pos.copy(), pos.copy()
+            pp[a, c] += h
+            pm[a, c] -= h
+            fdp[a, c] = (_loss(model, pp, x, nbr, mask, g) - _loss(model, pm, x, nbr, mask, g)) / (2 * h)
+    assert np.linalg.norm(gx - fdx) <= 1e-7 * np.linalg.norm(fdx)
+    assert np.linalg.norm(gpos - fdp) <= 1e-7 * np.linalg.norm(fdp)
+
+
+def test_attention_vjp_invariances_and_rows(attn_system):
+    model, pos, x, nbr, mask, g = attn_system
+    gx, gpos = oracle.attention_vjp(model, pos, nbr, mask, x, g)
+    scale = np.abs(gpos).max()
+    assert np.abs(gpos.sum(axis=0)).max() <= 1e-12 * scale * len(pos)  # translation invariance
+    # the gradient at atom k needs only the rows that read k: k itself and the rows listing k
+    k = 5
+    rows = sorted({k} | {i for i in range(len(pos)) if np.any((nbr[i] == k) & (mask[i] != 0))})
+    gx_k, gpos_k = oracle.attention_vjp(model, pos, nbr, mask, x, g, rows=rows)
+    assert np.allclose(gx_k[k], gx[k], rtol=1e-12, atol=1e-14)
+    assert np.allclose(gpos_k[k], gpos[k], rtol=1e-12, atol=1e-14)
+
+
+def test_attention_vjp_single_neighbor_by_hand():
+    """One valid slot per row: alpha = 1, so the logits carry no gradient and dL/dx_j is the sum of
+    g_i (.) W(d_ij) over the rows i that list j."""
+    model, w, wl = small_model(F=4, R=5, n_heads=2, head_dim=2)
+    pos = np.array([[0, 0, 0], [1.5, 0.5, 0], [0, 2.5, 1.0]], dtype=np.float64)
+    x = synth.node_features(3, 4, seed=6).astype(np.float64)
+    nbr = np.array([[1, -1], [0, -1], [0, -1]], dtype=np.int32)
+    mask = (nbr >= 0).astype(np.uint8)
+    g = np.random.default_rng(3).normal(size=(3, 4))
+    gx, gpos = oracle.attention_vjp(model, pos, nbr, mask, x, g)
+    W10 = oracle.filter_weights(model, 0, np.array([np.linalg.norm(pos[1] - pos[0])]))[0]
+    W20 = oracle.filter_weights(model, 0, np.array([np.linalg.norm(pos[2] - pos[0])]))[0]
+    assert np.allclose(gx[0], g[1] * W10 + g[2] * W20, rtol=1e-12)
+    assert np.allclose(gx[1], g[0] * W10, rtol=1e-12)
+    assert np.allclose(gx[2], 0.0)
+
+
 # ----------------------------------------------------------------------------- molecular dynamics
 def test_verlet_free_flight_is_exact():
     rng = np.random.default_rng(0)
