@@ -14,7 +14,7 @@ const char* kernel_name(int id) {
   static const char* names[K_NUM] = {
       "embed", "dense", "readout_energy", "readout_bwd", "graph_energy_sum", "cfconv_fwd_simt",
       "cfconv_bwd_simt", "attn_simt", "validate_csr", "cfconv_fwd_tc", "cfconv_bwd_tc",
-      "attn_tc", "dense_tc", "md_integrate"};
+      "attn_tc", "dense_tc", "md_integrate", "attn_bwd"};
   return (id >= 0 && id < K_NUM) ? names[id] : "?";
 }
 
@@ -172,6 +172,13 @@ extern "C" int mp_init(mp_ctx** out_ctx, const mp_config* cfg, const mp_weights*
   }
   extra.push_back(transpose(host[1 + (size_t)B * 8], F, Fh));
   extra_dst.push_back(&c->B1T);
+  if (H > 0) {  // the attention backward's dL/dx = dL/dq Wq^T + dL/dk Wk^T
+    const size_t qi = 1 + (size_t)B * 8 + 4;
+    extra.push_back(transpose(host[qi], F, F));
+    extra_dst.push_back(&c->WqT);
+    extra.push_back(transpose(host[qi + 1], F, F));
+    extra_dst.push_back(&c->WkT);
+  }
 
   size_t total = 0;
   for (auto& h : host) total += align_up(h.size() * sizeof(float), 256);
@@ -210,7 +217,8 @@ extern "C" int mp_init(mp_ctx** out_ctx, const mp_config* cfg, const mp_weights*
                     nf * st,           // g_m
                     nf * 4,            // grad_h
                     nf * 4, nf * 4,    // q, k
-                    N * 3 * 4};        // md_ref
+                    N * 3 * 4,         // md_ref
+                    N * 3 * (size_t)(H > 0 ? H : 1) * 4};  // attn_stats
   size_t ws = 0;
   for (size_t v : sizes) ws += align_up(v, 256);
   char* wsb = nullptr;
@@ -237,6 +245,7 @@ extern "C" int mp_init(mp_ctx** out_ctx, const mp_config* cfg, const mp_weights*
   c->q = (float*)take(sizes[9]);
   c->k = (float*)take(sizes[10]);
   c->md_ref = (float*)take(sizes[11]);
+  c->attn_stats = (float*)take(sizes[12]);
   if (cudaMalloc(&c->status_d, 4 * sizeof(int)) != cudaSuccess ||
       cudaMallocHost(&c->status_h, 4 * sizeof(int)) != cudaSuccess) {
     free_ctx(c);

@@ -34,7 +34,7 @@ struct FilterW {
 enum KernelId : int {
   K_EMBED = 0, K_DENSE, K_READOUT_E, K_READOUT_BWD, K_GRAPH_SUM, K_CFCONV_FWD_SIMT,
   K_CFCONV_BWD_SIMT, K_ATTN_SIMT, K_VALIDATE, K_CFCONV_FWD_TC, K_CFCONV_BWD_TC, K_ATTN_TC,
-  K_DENSE_TC, K_MD, K_NUM
+  K_DENSE_TC, K_MD, K_ATTN_BWD, K_NUM
 };
 const char* kernel_name(int id);
 
@@ -71,6 +71,8 @@ struct mp_ctx {
   float* q = nullptr;                     // [N][F] attention queries
   float* k = nullptr;                     // [N][F] attention keys
   float* md_ref = nullptr;                // [N][3] positions at the last neighbor-list build
+  float* attn_stats = nullptr;            // [N][3H] attention backward: row max, sum, g . out
+  float *WqT = nullptr, *WkT = nullptr;   // [F][F] transposed attention projections
   int* status_d = nullptr;                // device status bits (then the MD displacement flag)
   int* status_h = nullptr;                // pinned host copy
   int* md_flag = nullptr;                 // status_d + 1: an atom moved past the rebuild limit
@@ -178,6 +180,10 @@ int launch_attn_simt(mp_ctx*, int N, int K, const float* pos, const int* nbr,
                      const unsigned char* mask, const void* x, void* out, cudaStream_t);
 int launch_validate_csr(mp_ctx*, int N, long long E, const int* row_ptr, const int* col_idx,
                         const int* graph_ptr, int n_graphs, bool need_sym, cudaStream_t);
+// In place on the stream: a[1..n] counts -> a[0..n] prefix sums (a[0] = 0); *overflow = 1 when the
+// total passes INT_MAX. bsum: scan_blocks(n) (at least 1) long longs of scratch (neighbors.cu).
+int scan_blocks(long long n);
+void launch_scan(long long n, int* a, long long* bsum, int* overflow, cudaStream_t s);
 // The kernel sequence of one energy + forces evaluation (mp_api.cu), without validation or graphs.
 int energy_forces_launches(mp_ctx*, int N, long long E, const float* pos, const int* types,
                            const int* row_ptr, const int* col_idx, const int* graph_ptr,

@@ -134,6 +134,8 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_add(long long n, int* __r
   if (blockIdx.x == 0 && threadIdx.x == 0) a[0] = 0;
 }
 
+}  // namespace
+
 int scan_blocks(long long n) { return (int)((n + kScanPer - 1) / kScanPer); }
 
 // bsum: scan_blocks(n) (at least 1) long longs of scratch
@@ -147,6 +149,8 @@ void launch_scan(long long n, int* a, long long* bsum, int* overflow, cudaStream
   k_scan_totals<<<1, kScanThreads, 0, s>>>(nb, bsum, overflow);
   k_scan_add<<<nb, kScanThreads, 0, s>>>(n, a, bsum);
 }
+
+namespace {
 
 // ------------------------------------------------------------------------------------ cells
 struct CellGrid {

@@ -68,6 +68,7 @@ def _load():
         "mp_set_graphs": (i32, [vp, i32]),
         "mp_md_verlet": (i32, [vp, i32, i64, vp, vp, vp, vp, c_float, i32, vp, vp, vp, vp, i32,
                                vp, vp, vp]),
+        "mp_attn_bwd": (i32, [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp]),
         "mp_md_run": (i32, [vp, i32, vp, vp, vp, vp, c_float, i32, vp, vp, i32, c_float, i32,
                             c_float, i32, vp, vp, i64, POINTER(i64), vp, vp, POINTER(i32), vp]),
         "mp_selftest_tc": (i32, [POINTER(i32)]),
@@ -87,7 +88,7 @@ EXPORTED = ("mp_init", "mp_destroy", "mp_strerror", "mp_status_sync", "mp_neighb
             "mp_neighbor_padded", "mp_cfconv_fwd", "mp_attn_fwd", "mp_energy_forces",
             "mp_profile_begin", "mp_profile_end", "mp_profile_get", "mp_launch_count",
             "mp_attn_fwd_noalloc", "mp_selftest_tc", "mp_set_graphs",
-            "mp_md_verlet", "mp_md_run")
+            "mp_md_verlet", "mp_md_run", "mp_attn_bwd")
 NOALLOC_MAX_NF = 524288  # MP_NOALLOC_MAX_NF: largest N * F mp_attn_fwd_noalloc accepts
 
 
@@ -209,6 +210,25 @@ class Context:
         _check(lib.mp_attn_fwd(self._ctx, N, K, _ptr(pos), _ptr(nbr), _ptr(mask), _ptr(x),
                                _ptr(out), _stream(stream)), "mp_attn_fwd")
         return out
+
+    def attn_bwd(self, pos, nbr, mask, x, g_out, grad_x=None, grad_pos=None, stream=None):
+        """mp_attn_bwd: (dL/dx, dL/dpos) of L = sum g_out . attn_fwd(...), both float32."""
+        N, K = nbr.shape
+        _need(pos, "pos", torch.float32, (N, 3))
+        _need(nbr, "nbr", torch.int32, (N, K))
+        _need(mask, "mask", torch.uint8, (N, K))
+        _need(x, "x", self.tdtype, (N, self.F))
+        _need(g_out, "g_out", torch.float32, (N, self.F))
+        if grad_x is None:
+            grad_x = torch.empty((N, self.F), dtype=torch.float32, device=pos.device)
+        if grad_pos is None:
+            grad_pos = torch.empty((N, 3), dtype=torch.float32, device=pos.device)
+        _need(grad_x, "grad_x", torch.float32, (N, self.F))
+        _need(grad_pos, "grad_pos", torch.float32, (N, 3))
+        _check(lib.mp_attn_bwd(self._ctx, N, K, _ptr(pos), _ptr(nbr), _ptr(mask), _ptr(x),
+                               _ptr(g_out), _ptr(grad_x), _ptr(grad_pos), _stream(stream)),
+               "mp_attn_bwd")
+        return grad_x, grad_pos
 
     def energy_forces(self, pos, types, row_ptr, col_idx, graph_ptr=None, energy=None,
                       forces=None, stream=None):

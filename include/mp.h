@@ -162,6 +162,21 @@ int mp_cfconv_fwd(mp_ctx* ctx, int block, int N, long long E, const float* pos,
 int mp_attn_fwd(mp_ctx* ctx, int N, int K, const float* pos, const int* nbr,
                 const unsigned char* mask, const void* x, void* out, void* stream);
 
+/* Backward of mp_attn_fwd [E2 s.3.2; TS forces are position gradients]: for L = sum_i g_out_i .
+ * out_i, returns grad_x = dL/dx (float32 [N][F]) and grad_pos = dL/dr (float32 [N][3]; the
+ * forces are -grad_pos when L is an energy), through q, k, the radial logit bias, the filter
+ * W(d) and its envelope. Same nbr / mask / x conventions as mp_attn_fwd; g_out float32 [N][F].
+ * Two passes without atomics: per destination row (softmax statistics, dL/dq, the row-side
+ * position terms), then per source atom over the transposed list (dL/dk, the value path, the
+ * source-side position terms); deterministic. Needs n_heads * head_dim = F, n_heads <= 32,
+ * head_dim dividing 32, and 16 K n_heads + 16 K bytes of per-row slot data on chip beside the
+ * filter weights (K <= 256 at F = 128, n_rbf = 50, 16 heads), else MP_ERR_CAPACITY; N K < 2^31.
+ * Allocates and frees O(N K) bytes of stream-ordered scratch (the transposed list).
+ * Errors: MP_ERR_INVALID_ARG, MP_ERR_CAPACITY, MP_ERR_CUDA.                                    */
+int mp_attn_bwd(mp_ctx* ctx, int N, int K, const float* pos, const int* nbr,
+                const unsigned char* mask, const void* x, const float* g_out, float* grad_x,
+                float* grad_pos, void* stream);
+
 /* Allocation-free attention aggregation (no counterpart in the paper; added for callers that
  * cannot allocate device memory). Some hosts own every byte of device memory through their own
  * pool or budget and hand a library only pre-allocated buffers -- an MD engine's plugin

@@ -1,0 +1,103 @@
+"""Attention backward (dL/dx, dL/dr of L = sum g . out) through mp_attn_bwd vs the fp64 oracle's
+reverse-mode formulas (pinned by central differences), on seeded inputs: element by element at
+sizes spanning several batches and rows with capped lists, and on sampled atoms at the full
+attention workload (32,768 atoms, K = 256), where the oracle needs only the rows that read an atom.
+
+Tolerance: the kernels compute in fp32 from the stored inputs (bf16 features under a bf16
+context), so the bound is an fp32 one on both paths: normwise max|d| / max|ref| <= 1e-4. The
+gradients sum O(K) terms per row and O(K) entries per source of mixed sign, so cancellation
+costs about two decimal digits over the fp32 feature bound of 1e-5."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from atomistic_neighbor_list_b200 import synth
+from helpers import features_for, normwise, oracle_padded, oracle_weights
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+TOL = 1e-4
+
+
+@pytest.fixture(scope="module")
+def mp(cuda_ok):
+    from atomistic_neighbor_list_b200 import mp as m
+    return m
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+
+
+def case(mp, n, K, r_c, dtype, seed=0):
+    wl = dataclasses.replace(synth.WORKLOADS["cfg4"], n_atoms=n, K=K, dtype=dtype, r_c=r_c)
+    pos = synth.uniform_positions(n, seed=seed)
+    w = synth.make_weights(wl)
+    nbr, mask = mp.neighbor_padded(dev(pos), wl.r_c, K)
+    onbr, omask = oracle_padded(pos, wl.r_c, K, nbr, mask)
+    ctx = mp.Context.from_workload(wl, w, max_atoms=n, max_edges=1)
+    x_t, x_ref = features_for(synth.node_features(n, wl.F, seed=seed + 3), dtype)
+    g = np.random.default_rng(seed + 11).normal(size=(n, wl.F)).astype(np.float32)
+    model = oracle.Model.from_workload(wl, oracle_weights(w, dtype))
+    return wl, pos, nbr, mask, onbr, omask, ctx, x_t, x_ref, g, model
+
+
+@pytest.mark.parametrize("n,K,r_c,dtype", [(600, 20, 5.0, "fp32"), (1500, 64, 6.0, "fp32"),
+                                           (1200, 48, 5.0, "bf16"), (300, 16, 8.5, "fp32")])
+def test_attn_bwd_matches_oracle(mp, n, K, r_c, dtype):
+    wl, pos, nbr, mask, onbr, omask, ctx, x_t, x_ref, g, model = case(mp, n, K, r_c, dtype)
+    gx, gp = ctx.attn_bwd(dev(pos), nbr, mask, x_t.to(DEV), dev(g))
+    torch.cuda.synchronize()
+    ctx.status_sync()
+    rgx, rgp = oracle.attention_vjp(model, pos, onbr, omask, x_ref, g.astype(np.float64))
+    assert normwise(gx.cpu().numpy(), rgx) <= TOL
+    assert normwise(gp.cpu().numpy(), rgp) <= TOL
+    # translation invariance of L: the position gradients sum to zero
+    s = gp.double().sum(dim=0).abs().max().item()
+    assert s <= 1e-5 * gp.abs().sum().item()
+
+
+def test_attn_bwd_deterministic_and_empty_rows(mp):
+    """Rows without valid slots contribute nothing; two runs give the same bits."""
+    wl, pos, nbr, mask, onbr, omask, ctx, x_t, x_ref, g, model = case(mp, 400, 12, 5.0, "fp32", 2)
+    omask = omask.copy()
+    omask[::7] = 0  # every 7th row has no valid slot
+    nbr, mask = dev(onbr), dev(omask)
+    a = ctx.attn_bwd(dev(pos), nbr, mask, x_t.to(DEV), dev(g))
+    b = ctx.attn_bwd(dev(pos), nbr, mask, x_t.to(DEV), dev(g))
+    torch.cuda.synchronize()
+    ctx.status_sync()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    rgx, rgp = oracle.attention_vjp(model, pos, onbr, omask, x_ref, g.astype(np.float64))
+    assert normwise(a[0].cpu().numpy(), rgx) <= TOL
+    assert normwise(a[1].cpu().numpy(), rgp) <= TOL
+
+
+def test_attn_bwd_full_size_sampled(mp):
+    """32,768 atoms, K = 256, bf16: sampled atoms against the oracle restricted to the rows that
+    read them (the gradient at atom k depends on row k and the rows listing k only)."""
+    wl = synth.WORKLOADS["cfg4"]
+    n, K = wl.n_atoms, wl.K
+    pos = synth.uniform_positions(n, seed=0)
+    w = synth.make_weights(wl)
+    nbr, mask = mp.neighbor_padded(dev(pos), wl.r_c, K)
+    ctx = mp.Context.from_workload(wl, w, max_atoms=n, max_edges=1)
+    x_t, x_ref = features_for(synth.node_features(n, wl.F), wl.dtype)
+    g = np.random.default_rng(11).normal(size=(n, wl.F)).astype(np.float32)
+    gx, gp = ctx.attn_bwd(dev(pos), nbr, mask, x_t.to(DEV), dev(g))
+    torch.cuda.synchronize()
+    ctx.status_sync()
+    gx, gp = gx.cpu().numpy(), gp.cpu().numpy()
+    assert np.all(np.isfinite(gx)) and np.all(np.isfinite(gp))
+    assert np.abs(gp.astype(np.float64).sum(axis=0)).max() <= 1e-5 * np.abs(gp).sum()
+    onbr, omask = oracle_padded(pos, wl.r_c, K, nbr, mask)
+    model = oracle.Model.from_workload(wl, oracle_weights(w, wl.dtype))
+    for k in (0, 12345, n // 2 + 77, n - 1):
+        rows = sorted({k} | set(np.nonzero(np.any((onbr == k) & (omask != 0), axis=1))[0].tolist()))
+        rgx, rgp = oracle.attention_vjp(model, pos, onbr, omask, x_ref, g.astype(np.float64),
+                                        rows=rows)
+        assert np.abs(gx[k] - rgx[k]).max() <= TOL * np.abs(rgx[k]).max() * 10
+        assert np.linalg.norm(gp[k] - rgp[k]) <= TOL * 10 * np.linalg.norm(rgp[k])
