@@ -24,19 +24,23 @@ constexpr int AB = 16;  // entries per batch
 
 template <int F>
 struct AbSmem {
-  float rbf[kMaxR][AB], drbf[kMaxR][AB];
-  float h1[F][AB + 1], h1p[F][AB + 1];
+  // rows of AB entries, read as float4 (one load serves four entries' FMAs)
+  __align__(16) float rbf[kMaxR][AB];
+  __align__(16) float drbf[kMaxR][AB];
+  __align__(16) float h1[F][AB];
+  __align__(16) float h1p[F][AB];
   int src[AB], dst[AB], ok[AB];
   float d[AB], fc[AB], dfc[AB], u[AB][3];
   float spart[AB][32];  // per entry and head: alpha beta + dl b' (source pass)
+  float st[AB][3 * 32];  // per entry: its row's softmax statistics (source pass)
   float red[3][F / 32];
 };
 
 // Filter W and dW/dd of the batch's entries for feature f (every thread of the CTA calls it;
 // s.d / s.fc / s.dfc / s.ok set for t < nb). Identical arithmetic in both passes.
 template <int F>
-__device__ __forceinline__ void filter_batch(AbSmem<F>& s, int nb, const float* __restrict__ sA1,
-                                             const float* __restrict__ sA2, float c1f, float c2f,
+__device__ __forceinline__ void filter_batch(AbSmem<F>& s, int nb, const float* __restrict__ A1,
+                                             const float* __restrict__ A2, float c1f, float c2f,
                                              const Radial& rp, float (&W)[AB], float (&Wp)[AB]) {
   const int f = threadIdx.x;
   for (int idx = f; idx < rp.R * AB; idx += F) {
@@ -54,17 +58,30 @@ __device__ __forceinline__ void filter_batch(AbSmem<F>& s, int nb, const float* 
     tz[t] = 0.f;
   }
   for (int k = 0; k < rp.R; ++k) {
-    const float a = sA1[k * F + f];
+    const float a = __ldg(A1 + k * F + f);
 #pragma unroll
-    for (int t = 0; t < AB; ++t) {
-      z[t] = fmaf(s.rbf[k][t], a, z[t]);
-      tz[t] = fmaf(s.drbf[k][t], a, tz[t]);
+    for (int t4 = 0; t4 < AB; t4 += 4) {
+      const float4 e = *(const float4*)&s.rbf[k][t4];
+      const float4 de = *(const float4*)&s.drbf[k][t4];
+      z[t4] = fmaf(e.x, a, z[t4]);
+      z[t4 + 1] = fmaf(e.y, a, z[t4 + 1]);
+      z[t4 + 2] = fmaf(e.z, a, z[t4 + 2]);
+      z[t4 + 3] = fmaf(e.w, a, z[t4 + 3]);
+      tz[t4] = fmaf(de.x, a, tz[t4]);
+      tz[t4 + 1] = fmaf(de.y, a, tz[t4 + 1]);
+      tz[t4 + 2] = fmaf(de.z, a, tz[t4 + 2]);
+      tz[t4 + 3] = fmaf(de.w, a, tz[t4 + 3]);
     }
   }
+  // thread f's row of AB values as float4 stores (the lanes of a warp conflict on these 64-byte
+  // rows, but each row is written once per batch and read 4 x F times)
 #pragma unroll
-  for (int t = 0; t < AB; ++t) {
-    s.h1[f][t] = ssp_f(z[t]);
-    s.h1p[f][t] = sigmoid_f(z[t]) * tz[t];
+  for (int t4 = 0; t4 < AB; t4 += 4) {
+    *(float4*)&s.h1[f][t4] = make_float4(ssp_f(z[t4]), ssp_f(z[t4 + 1]), ssp_f(z[t4 + 2]),
+                                         ssp_f(z[t4 + 3]));
+    *(float4*)&s.h1p[f][t4] =
+        make_float4(sigmoid_f(z[t4]) * tz[t4], sigmoid_f(z[t4 + 1]) * tz[t4 + 1],
+                    sigmoid_f(z[t4 + 2]) * tz[t4 + 2], sigmoid_f(z[t4 + 3]) * tz[t4 + 3]);
   }
   __syncthreads();
   float u[AB], up[AB];
@@ -74,11 +91,19 @@ __device__ __forceinline__ void filter_batch(AbSmem<F>& s, int nb, const float* 
     up[t] = 0.f;
   }
   for (int g = 0; g < F; ++g) {
-    const float a = sA2[g * F + f];
+    const float a = __ldg(A2 + g * F + f);
 #pragma unroll
-    for (int t = 0; t < AB; ++t) {
-      u[t] = fmaf(s.h1[g][t], a, u[t]);
-      up[t] = fmaf(s.h1p[g][t], a, up[t]);
+    for (int t4 = 0; t4 < AB; t4 += 4) {
+      const float4 h = *(const float4*)&s.h1[g][t4];
+      const float4 hp = *(const float4*)&s.h1p[g][t4];
+      u[t4] = fmaf(h.x, a, u[t4]);
+      u[t4 + 1] = fmaf(h.y, a, u[t4 + 1]);
+      u[t4 + 2] = fmaf(h.z, a, u[t4 + 2]);
+      u[t4 + 3] = fmaf(h.w, a, u[t4 + 3]);
+      up[t4] = fmaf(hp.x, a, up[t4]);
+      up[t4 + 1] = fmaf(hp.y, a, up[t4 + 1]);
+      up[t4 + 2] = fmaf(hp.z, a, up[t4 + 2]);
+      up[t4 + 3] = fmaf(hp.w, a, up[t4 + 3]);
     }
   }
 #pragma unroll
@@ -130,8 +155,8 @@ __device__ __forceinline__ float bias_grad_part(const float (*drbf)[AB], int t,
 
 // ------------------------------------------------------------------------------ destination pass
 // One CTA (F threads, thread f = channel f of head f / D) per destination row. Dynamic shared
-// memory: A1 [R][F], A2 [F][F], P [R][H], then per slot: logit, dalpha, beta, b' ([K][H] each),
-// the unit vector [K][3] and the source [K].
+// memory per slot: logit, dalpha, beta, b' ([K][H] each), the unit vector [K][3] and the source
+// [K]; the filter weights are read through L1 (they stay resident: every CTA reads the same).
 template <typename T, int F>
 __global__ void __launch_bounds__(F) k_attn_bwd_dst(
     int N, int K, const float* __restrict__ pos, const int* __restrict__ nbr,
@@ -140,10 +165,8 @@ __global__ void __launch_bounds__(F) k_attn_bwd_dst(
     const float* __restrict__ P, const float* __restrict__ pb, int H, int D,
     float* __restrict__ gq, float* __restrict__ grad_pos, float* __restrict__ stats, int* status) {
   extern __shared__ float dsm[];
-  float* sA1 = dsm;
-  float* sA2 = sA1 + rp.R * F;
-  float* sP = sA2 + F * F;
-  float* sl = sP + rp.R * H;
+  const float* sP = P;
+  float* sl = dsm;
   float* sda = sl + K * H;
   float* sbeta = sda + K * H;
   float* sbp = sbeta + K * H;
@@ -153,12 +176,8 @@ __global__ void __launch_bounds__(F) k_attn_bwd_dst(
 
   const int f = threadIdx.x, lane = f & 31, warp = f >> 5;
   const int head = f / D, c = f % D;
-  for (int i = f; i < rp.R * F; i += F) sA1[i] = fw.A1[i];
-  for (int i = f; i < F * F; i += F) sA2[i] = fw.A2[i];
-  for (int i = f; i < rp.R * H; i += F) sP[i] = P[i];
   const float c1f = fw.c1[f], c2f = fw.c2[f];
   const float inv_sqrt_d = rsqrtf((float)D);
-  __syncthreads();
 
   for (int i = blockIdx.x; i < N; i += gridDim.x) {
     const float qi = q[(size_t)i * F + f] * inv_sqrt_d;
@@ -192,14 +211,20 @@ __global__ void __launch_bounds__(F) k_attn_bwd_dst(
       }
       __syncthreads();
       float W[AB], Wp[AB];
-      filter_batch<F>(s, nb, sA1, sA2, c1f, c2f, rp, W, Wp);
+      filter_batch<F>(s, nb, fw.A1, fw.A2, c1f, c2f, rp, W, Wp);
+      // the batch's row gathers issued together (s.src is 0 for empty entries: always in range)
+      float xr[AB], kr[AB];
+#pragma unroll
+      for (int t = 0; t < AB; ++t) {
+        xr[t] = ldf(x + (size_t)s.src[t] * F + f);
+        kr[t] = kx[(size_t)s.src[t] * F + f];
+      }
 #pragma unroll
       for (int t = 0; t < AB; ++t) {
         if (t < nb && s.ok[t]) {  // uniform across the CTA
-          const int j = s.src[t];
-          const float xj = ldf(x + (size_t)j * F + f);
-          const float l = head_sum(logit_part(qi, kx[(size_t)j * F + f], s.rbf, t, sP, rp.R, H,
-                                              head, c, D), D) + pb[head];
+          const float xj = xr[t];
+          const float l = head_sum(logit_part(qi, kr[t], s.rbf, t, sP, rp.R, H, head, c, D), D) +
+                          pb[head];
           const float da = head_sum(gi * xj * W[t], D);
           const float be = head_sum(gi * xj * Wp[t], D);
           const float bp = head_sum(bias_grad_part(s.drbf, t, sP, rp.R, H, head, c, D), D);
@@ -235,12 +260,22 @@ __global__ void __launch_bounds__(F) k_attn_bwd_dst(
     }
     // dL/dq_i: every valid slot's dl times k_j
     float acc = 0.f;
-    for (int sl0 = 0; sl0 < K; ++sl0) {
-      const int j = ssrc[sl0];
-      if (j < 0) continue;  // uniform
-      const int o = sl0 * H + head;
-      const float a = expf(sl[o] - m) * iz;
-      acc = fmaf(a * (sda[o] - Dh), kx[(size_t)j * F + f], acc);
+    for (int b0 = 0; b0 < K; b0 += 8) {  // eight independent gathers in flight
+      float kv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j = b0 + u < K ? ssrc[b0 + u] : -1;
+        kv[u] = j >= 0 ? kx[(size_t)j * F + f] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int sl0 = b0 + u;
+        if (sl0 < K && ssrc[sl0] >= 0) {  // uniform
+          const int o = sl0 * H + head;
+          const float a = expf(sl[o] - m) * iz;
+          acc = fmaf(a * (sda[o] - Dh), kv[u], acc);
+        }
+      }
     }
     gq[(size_t)i * F + f] = acc * inv_sqrt_d;
     // dL/dr_i: each slot's dL/dd summed over the heads (thread f takes slots f, f + F, ...)
@@ -293,20 +328,13 @@ __global__ void __launch_bounds__(F) k_attn_bwd_src(
     const float* __restrict__ P, const float* __restrict__ pb, int H, int D,
     const float* __restrict__ stats, float* __restrict__ grad_x, float* __restrict__ gk,
     float* __restrict__ grad_pos, int* status) {
-  extern __shared__ float dsm[];
-  float* sA1 = dsm;
-  float* sA2 = sA1 + rp.R * F;
-  float* sP = sA2 + F * F;
+  const float* sP = P;
   __shared__ AbSmem<F> s;
 
   const int f = threadIdx.x, lane = f & 31, warp = f >> 5;
   const int head = f / D, c = f % D;
-  for (int i = f; i < rp.R * F; i += F) sA1[i] = fw.A1[i];
-  for (int i = f; i < F * F; i += F) sA2[i] = fw.A2[i];
-  for (int i = f; i < rp.R * H; i += F) sP[i] = P[i];
   const float c1f = fw.c1[f], c2f = fw.c2[f];
   const float inv_sqrt_d = rsqrtf((float)D);
-  __syncthreads();
 
   for (int j = blockIdx.x; j < N; j += gridDim.x) {
     const int r0 = rev_ptr[j], r1 = rev_ptr[j + 1];
@@ -330,6 +358,8 @@ __global__ void __launch_bounds__(F) k_attn_bwd_src(
             i = 0;
           }
         }
+        if (ok)
+          for (int k = 0; k < 3 * H; ++k) s.st[t][k] = stats[(size_t)i * 3 * H + k];
         s.dst[t] = i;
         s.ok[t] = ok;
         s.d[t] = d;
@@ -341,14 +371,19 @@ __global__ void __launch_bounds__(F) k_attn_bwd_src(
       }
       __syncthreads();
       float W[AB], Wp[AB];
-      filter_batch<F>(s, nb, sA1, sA2, c1f, c2f, rp, W, Wp);
+      filter_batch<F>(s, nb, fw.A1, fw.A2, c1f, c2f, rp, W, Wp);
+      float qr[AB], gr[AB];  // the batch's row gathers issued together (s.dst is 0 when empty)
+#pragma unroll
+      for (int t = 0; t < AB; ++t) {
+        qr[t] = q[(size_t)s.dst[t] * F + f];
+        gr[t] = g[(size_t)s.dst[t] * F + f];
+      }
 #pragma unroll
       for (int t = 0; t < AB; ++t) {
         if (t < nb && s.ok[t]) {  // uniform across the CTA
-          const int i = s.dst[t];
-          const float qi = q[(size_t)i * F + f] * inv_sqrt_d;
-          const float gi = g[(size_t)i * F + f];
-          const float* st = stats + (size_t)i * 3 * H;
+          const float qi = qr[t] * inv_sqrt_d;
+          const float gi = gr[t];
+          const float* st = s.st[t];
           const float l = head_sum(logit_part(qi, kj, s.rbf, t, sP, rp.R, H, head, c, D), D) +
                           pb[head];
           const float z = st[H + head];
@@ -432,9 +467,7 @@ int run_attn_bwd(mp_ctx* c, int N, int K, const float* pos, const int* nbr,
                  const unsigned char* mask, const void* x, const float* g, float* grad_x,
                  float* grad_pos, const int* rev_ptr, const int* rev, cudaStream_t s) {
   const int H = c->cfg.n_heads, D = c->cfg.head_dim, R = c->cfg.n_rbf;
-  const size_t w_floats = (size_t)R * F + (size_t)F * F + (size_t)R * H;
-  const size_t smem_dst = (w_floats + 4 * (size_t)K * H + 3 * (size_t)K) * 4 + (size_t)K * 4;
-  const size_t smem_src = w_floats * 4;
+  const size_t smem_dst = (4 * (size_t)K * H + 3 * (size_t)K) * 4 + (size_t)K * 4;
   auto kd = k_attn_bwd_dst<T, F>;
   auto ks = k_attn_bwd_src<T, F>;
   int optin = 0;
@@ -445,21 +478,25 @@ int run_attn_bwd(mp_ctx* c, int N, int K, const float* pos, const int* nbr,
     return MP_ERR_CUDA;
   if (fa.sharedSizeBytes + smem_dst > (size_t)optin) return MP_ERR_CAPACITY;
   if (cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dst) !=
-          cudaSuccess ||
-      cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_src) !=
-          cudaSuccess) {
+      cudaSuccess) {
     cudaGetLastError();
     return MP_ERR_CAPACITY;  // K too large for the per-slot arrays on chip
   }
-  const int grid = N < 2 * c->num_sms ? (N > 0 ? N : 1) : 2 * c->num_sms;
+  // as many resident CTAs as fit, every SM busy (rows and sources are independent work items)
+  int occ_d = 1, occ_s = 1;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_d, kd, F, smem_dst);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_s, ks, F, 0);
+  const long long cap_d = (long long)c->num_sms * (occ_d > 0 ? occ_d : 1);
+  const long long cap_s = (long long)c->num_sms * (occ_s > 0 ? occ_s : 1);
+  const int grid_d = (int)(N < cap_d ? N : cap_d), grid_s = (int)(N < cap_s ? N : cap_s);
   float* gq = c->g_x;     // [N][F] scratch: dL/dq
   float* gk = c->grad_h;  // [N][F] scratch: dL/dk
-  int rc = launch(c, K_ATTN_BWD, kd, dim3(grid), dim3(F), smem_dst, s, N, K, pos, nbr, mask,
+  int rc = launch(c, K_ATTN_BWD, kd, dim3(grid_d), dim3(F), smem_dst, s, N, K, pos, nbr, mask,
                   (const T*)x, g, (const float*)c->q, (const float*)c->k, filter_of(c, 0),
                   radial_of(c), (const float*)c->P, (const float*)c->p, H, D, gq, grad_pos,
                   c->attn_stats, c->status_d);
   if (rc == MP_OK)
-    rc = launch(c, K_ATTN_BWD, ks, dim3(grid), dim3(F), smem_src, s, N, K, pos, rev_ptr, rev,
+    rc = launch(c, K_ATTN_BWD_SRC, ks, dim3(grid_s), dim3(F), 0, s, N, K, pos, rev_ptr, rev,
                 (const T*)x, g, (const float*)c->q, (const float*)c->k, filter_of(c, 0),
                 radial_of(c), (const float*)c->P, (const float*)c->p, H, D,
                 (const float*)c->attn_stats, grad_x, gk, grad_pos, c->status_d);
@@ -509,14 +546,14 @@ extern "C" int mp_attn_bwd(mp_ctx* c, int N, int K, const float* pos, const int*
   cudaMemsetAsync(rev_ptr, 0, 4 * ((size_t)N + 1 + (size_t)N), s);
   cudaMemsetAsync(overflow, 0, 4, s);
   const int eb = (int)((NK + 255) / 256);
-  rc = launch(c, K_ATTN_BWD, k_rev_count, dim3(eb), dim3(256), 0, s, N, K, nbr, mask, rev_ptr);
+  rc = launch(c, K_ATTN_REV, k_rev_count, dim3(eb), dim3(256), 0, s, N, K, nbr, mask, rev_ptr);
   if (rc == MP_OK) {
     launch_scan(N, rev_ptr, bsum, overflow, s);
-    rc = launch(c, K_ATTN_BWD, k_rev_fill, dim3(eb), dim3(256), 0, s, N, K, nbr, mask,
+    rc = launch(c, K_ATTN_REV, k_rev_fill, dim3(eb), dim3(256), 0, s, N, K, nbr, mask,
                 (const int*)rev_ptr, cursor, tmp);
   }
   if (rc == MP_OK)
-    rc = launch(c, K_ATTN_BWD, k_rev_sort, dim3(c->num_sms * 8), dim3(256), 0, s, N,
+    rc = launch(c, K_ATTN_REV, k_rev_sort, dim3(c->num_sms * 8), dim3(256), 0, s, N,
                 (const int*)rev_ptr, (const int*)tmp, rev);
   if (rc == MP_OK) {
     if (F == 64)

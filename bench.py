@@ -377,6 +377,26 @@ def main():
         ms4 = sum(a.elapsed_time(b) for a, b in ev4) / len(ev4)
         attn = {"value": valid4 / (ms4 / 1000.0), "unit": "edges/s", "ms_per_call": ms4,
                 "workload": f"cfg4 ({n4} atoms, K={wl4.K}, {valid4} valid edges, {wl4.dtype})"}
+        # its backward (dL/dx and dL/dr for an upstream gradient), same timing rules
+        g4 = torch.randn((n4, wl4.F), generator=torch.Generator(device=devn).manual_seed(5),
+                         device=devn)
+        gx4 = torch.empty((n4, wl4.F), dtype=torch.float32, device=devn)
+        gp4 = torch.empty((n4, 3), dtype=torch.float32, device=devn)
+        ctx4.attn_bwd(pos4_d, nbr4, mask4, x4, g4, gx4, gp4)
+        evb = []
+        for _ in range(3):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            ctx4.attn_bwd(pos4_d, nbr4, mask4, x4, g4, gx4, gp4)
+            b.record(stream)
+            evb.append((a, b))
+        torch.cuda.synchronize()
+        ctx4.status_sync()
+        msb = sum(a.elapsed_time(b) for a, b in evb) / len(evb)
+        attn["backward"] = {"value": valid4 / (msb / 1000.0), "unit": "edges/s",
+                            "ms_per_call": msb, "path": "SIMT fp32 math, two passes"}
+        del g4, gx4, gp4
         ctx4.close()
         del nbr4, mask4, x4, o4, pos4_d
 
