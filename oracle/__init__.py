@@ -34,5 +34,7 @@ from .schnet import (  # noqa: F401
     LN2, rbf_centres, gaussian_rbf, gaussian_rbf_grad, cosine_cutoff, cosine_cutoff_grad, ssp,
     ssp_grad, filter_weights, cfconv, Model, energies, energy_forces,
 )
-from .attention import attention, attention_vjp  # noqa: F401
+from .attention import (  # noqa: F401
+    attention, attention_vjp, attention_equivariant, solid_harmonics, moments_to_solid,
+)
 from .md import kinetic_energy, velocity_verlet  # noqa: F401

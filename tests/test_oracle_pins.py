@@ -473,6 +473,78 @@ def test_attention_vjp_single_neighbor_by_hand():
     assert np.allclose(gx[2], 0.0)
 
 
+def test_solid_harmonics_match_library_real_sph_harm():
+    """Unit vectors: S_lm = Y_lm, the real form of scipy's complex harmonics (Condon-Shortley
+    phase): sqrt2 (-1)^m Re Y_l^m for m > 0, sqrt2 (-1)^m Im Y_l^|m| for m < 0; and S_lm is
+    homogeneous of degree l."""
+    import scipy.special as sp
+    rng = np.random.default_rng(0)
+    v = rng.normal(size=(200, 3))
+    v /= np.linalg.norm(v, axis=1)[:, None]
+    theta, phi = np.arccos(v[:, 2]), np.arctan2(v[:, 1], v[:, 0])
+    S = oracle.solid_harmonics(v)
+    col = 0
+    for l in range(3):
+        for m in range(-l, l + 1):
+            Y = sp.sph_harm_y(l, abs(m), theta, phi)
+            ref = Y.real if m == 0 else np.sqrt(2) * (-1) ** m * (Y.real if m > 0 else Y.imag)
+            assert np.allclose(S[:, col], ref, rtol=0, atol=1e-13), (l, m)
+            assert np.allclose(oracle.solid_harmonics(2.5 * v)[:, col], 2.5 ** l * S[:, col],
+                               rtol=1e-13, atol=1e-14)
+            col += 1
+
+
+def test_equivariant_attention_scalar_part_and_rotation(attn_system):
+    model, pos, x, nbr, mask, g = attn_system
+    out = oracle.attention_equivariant(model, pos, nbr, mask, x)
+    base = oracle.attention(model, pos, nbr, mask, x)
+    assert np.allclose(out[:, 0, :], base / (2 * math.sqrt(math.pi)), rtol=1e-12, atol=1e-14)
+    # rotate and translate the system: l = 1 rotates as a vector; each l block keeps its norm
+    rng = np.random.default_rng(4)
+    Q, _ = np.linalg.qr(rng.normal(size=(3, 3)))
+    if np.linalg.det(Q) < 0:
+        Q[:, 0] = -Q[:, 0]
+    pos_r = pos @ Q.T + np.array([3.0, -1.0, 7.0])
+    out_r = oracle.attention_equivariant(model, pos_r, nbr, mask, x)
+    vec = out[:, [3, 1, 2], :]      # (x, y, z) from the l = 1 components (y, z, x)
+    vec_r = out_r[:, [3, 1, 2], :]
+    assert np.allclose(np.einsum("ab,nbf->naf", Q, vec), vec_r, rtol=1e-10, atol=1e-12)
+    n2 = np.sum(out[:, 4:9, :] ** 2, axis=1)
+    n2_r = np.sum(out_r[:, 4:9, :] ** 2, axis=1)
+    assert np.allclose(n2, n2_r, rtol=1e-10, atol=1e-14)
+    assert np.allclose(out[:, 0], out_r[:, 0], rtol=1e-10, atol=1e-14)
+
+
+def test_equivariant_attention_node_centric_form(attn_system):
+    """E2Former-V2 section 3.1 in its node-centric form: couple each source's value with the
+    monomials of its own position, aggregate with the attention weights, then couple with the
+    destination's position. Equals the per-edge definition."""
+    model, pos, x, nbr, mask, g = attn_system
+    out = oracle.attention_equivariant(model, pos, nbr, mask, x)
+    w = model.w
+    H, D = model.n_heads, model.head_dim
+    n, K = nbr.shape
+    q, k = x @ w["Wq"], x @ w["Wk"]
+    mom = np.zeros((n, 10, x.shape[1]))
+    for i in range(n):
+        js = [int(nbr[i, s]) for s in range(K) if mask[i, s]]
+        if not js:
+            continue
+        d = np.linalg.norm(pos[js] - pos[i], axis=1)
+        e = oracle.gaussian_rbf(d, model.mu, model.gamma)
+        l = (np.einsum("hd,jhd->jh", q[i].reshape(H, D), k[js].reshape(-1, H, D)) / np.sqrt(D)
+             + e @ w["P"] + w["p"])
+        a = np.exp(l - l.max(axis=0))
+        a = np.repeat(a / a.sum(axis=0), D, axis=1)
+        v = a * x[js] * oracle.filter_weights(model, 0, d)          # alpha v, source values
+        X, Y, Z = pos[js, 0], pos[js, 1], pos[js, 2]                # source pre-coupling
+        mono = np.stack([np.ones_like(X), X, Y, Z, X * X, X * Y, X * Z, Y * Y, Y * Z, Z * Z], 1)
+        mom[i] = mono.T @ v
+    node = oracle.moments_to_solid(mom, pos)                        # target coupling
+    scale = np.abs(out).max()
+    assert np.abs(node - out).max() <= 1e-10 * scale
+
+
 # ----------------------------------------------------------------------------- molecular dynamics
 def test_verlet_free_flight_is_exact():
     rng = np.random.default_rng(0)
