@@ -69,6 +69,7 @@ def _load():
         "mp_md_verlet": (i32, [vp, i32, i64, vp, vp, vp, vp, c_float, i32, vp, vp, vp, vp, i32,
                                vp, vp, vp]),
         "mp_attn_bwd": (i32, [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "mp_attn_eq_fwd": (i32, [vp, i32, i32, vp, vp, vp, vp, vp, vp]),
         "mp_md_run": (i32, [vp, i32, vp, vp, vp, vp, c_float, i32, vp, vp, i32, c_float, i32,
                             c_float, i32, vp, vp, i64, POINTER(i64), vp, vp, POINTER(i32), vp]),
         "mp_selftest_tc": (i32, [POINTER(i32)]),
@@ -88,7 +89,7 @@ EXPORTED = ("mp_init", "mp_destroy", "mp_strerror", "mp_status_sync", "mp_neighb
             "mp_neighbor_padded", "mp_cfconv_fwd", "mp_attn_fwd", "mp_energy_forces",
             "mp_profile_begin", "mp_profile_end", "mp_profile_get", "mp_launch_count",
             "mp_attn_fwd_noalloc", "mp_selftest_tc", "mp_set_graphs",
-            "mp_md_verlet", "mp_md_run", "mp_attn_bwd")
+            "mp_md_verlet", "mp_md_run", "mp_attn_bwd", "mp_attn_eq_fwd")
 NOALLOC_MAX_NF = 524288  # MP_NOALLOC_MAX_NF: largest N * F mp_attn_fwd_noalloc accepts
 
 
@@ -209,6 +210,20 @@ class Context:
         _need(out, "out", self.tdtype, (N, self.F))
         _check(lib.mp_attn_fwd(self._ctx, N, K, _ptr(pos), _ptr(nbr), _ptr(mask), _ptr(x),
                                _ptr(out), _stream(stream)), "mp_attn_fwd")
+        return out
+
+    def attn_eq_fwd(self, pos, nbr, mask, x, out=None, stream=None):
+        """mp_attn_eq_fwd: [N, 9, F] equivariant attention values (solid harmonics l <= 2)."""
+        N, K = nbr.shape
+        _need(pos, "pos", torch.float32, (N, 3))
+        _need(nbr, "nbr", torch.int32, (N, K))
+        _need(mask, "mask", torch.uint8, (N, K))
+        _need(x, "x", self.tdtype, (N, self.F))
+        if out is None:
+            out = torch.empty((N, 9, self.F), dtype=self.tdtype, device=pos.device)
+        _need(out, "out", self.tdtype, (N, 9, self.F))
+        _check(lib.mp_attn_eq_fwd(self._ctx, N, K, _ptr(pos), _ptr(nbr), _ptr(mask), _ptr(x),
+                                  _ptr(out), _stream(stream)), "mp_attn_eq_fwd")
         return out
 
     def attn_bwd(self, pos, nbr, mask, x, g_out, grad_x=None, grad_pos=None, stream=None):

@@ -162,6 +162,20 @@ int mp_cfconv_fwd(mp_ctx* ctx, int block, int N, long long E, const float* pos,
 int mp_attn_fwd(mp_ctx* ctx, int N, int K, const float* pos, const int* nbr,
                 const unsigned char* mask, const void* x, void* out, void* stream);
 
+/* Neighbor attention with an equivariant value path [E2 s.3.1: direction enters only through
+ * the values]: the softmax weights of mp_attn_fwd, with each value coupled to the regular solid
+ * harmonics of the edge vector up to l = 2,
+ *   out_i[lm][c] = sum_j alpha_ij,h(c) (x_j (.) W(d_ij))[c] S_lm(r_j - r_i),
+ * S_lm(r) = |r|^l Y_lm(r / |r|) with Y the real spherical harmonics orthonormal on the sphere, in
+ * the order (l,m) = (0,0), (1,-1), (1,0), (1,1), (2,-2), (2,-1), (2,0), (2,1), (2,2); so
+ * out_i[0] = mp_attn_fwd(...)_i / (2 sqrt(pi)) and out_i[1..3] rotate as (y, z, x).
+ * out: [N][9][F] of the context dtype (device). The harmonics are evaluated per edge on chip
+ * (the page's node-centric factorisation through source and destination positions gives the same
+ * sum but loses digits to cancellation in fp32). Fp32 math on the CUDA cores. Same arguments,
+ * conventions and errors as mp_attn_fwd.                                                      */
+int mp_attn_eq_fwd(mp_ctx* ctx, int N, int K, const float* pos, const int* nbr,
+                   const unsigned char* mask, const void* x, void* out, void* stream);
+
 /* Backward of mp_attn_fwd [E2 s.3.2; TS forces are position gradients]: for L = sum_i g_out_i .
  * out_i, returns grad_x = dL/dx (float32 [N][F]) and grad_pos = dL/dr (float32 [N][3]; the
  * forces are -grad_pos when L is an energy), through q, k, the radial logit bias, the filter
