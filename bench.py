@@ -397,6 +397,23 @@ def main():
         attn["backward"] = {"value": valid4 / (msb / 1000.0), "unit": "edges/s",
                             "ms_per_call": msb, "path": "SIMT fp32 math, two passes"}
         del g4, gx4, gp4
+        # the equivariant value path (solid harmonics l <= 2 on each value), same timing rules
+        oe4 = torch.empty((n4, 9, wl4.F), dtype=x4.dtype, device=devn)
+        ctx4.attn_eq_fwd(pos4_d, nbr4, mask4, x4, oe4)
+        eve = []
+        for _ in range(3):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            ctx4.attn_eq_fwd(pos4_d, nbr4, mask4, x4, oe4)
+            b.record(stream)
+            eve.append((a, b))
+        torch.cuda.synchronize()
+        ctx4.status_sync()
+        mse = sum(a.elapsed_time(b) for a, b in eve) / len(eve)
+        attn["equivariant"] = {"value": valid4 / (mse / 1000.0), "unit": "edges/s",
+                               "ms_per_call": mse, "path": "SIMT fp32 math, l <= 2"}
+        del oe4
         ctx4.close()
         del nbr4, mask4, x4, o4, pos4_d
 
