@@ -50,6 +50,30 @@ def rank_info():
             int(os.environ.get("LOCAL_RANK", 0)))
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time: each rank passes its own device-timed milliseconds and every rank
+    gets the maximum (one all-reduce of a scalar; timing plumbing, not a data-path collective)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: each of `world` ranks ran `steps` steps of its own independent system
+    (weak scaling), and the job took as long as its slowest rank."""
+    return world * steps / (max_ms / 1000.0)
+
+
+def rank_system(wl, rank: int):
+    """The system rank `rank` simulates: the workload's generator seeded by the rank, so the
+    ranks run independent replicas of the same size (positions float32 [N,3], graph_ptr)."""
+    from atomistic_neighbor_list_b200 import synth
+    return synth.positions_for(wl, seed=rank)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -265,7 +289,7 @@ def main():
                                 device_id=torch.device(devn))
     peaks = load_peaks()
     wl = synth.WORKLOADS[args.workload]
-    pos, gp = synth.positions_for(wl, seed=rank)
+    pos, gp = rank_system(wl, rank)
     N = len(pos)
     types = synth.atom_types(N, wl.n_types)
     weights = synth.make_weights(wl)
@@ -315,11 +339,8 @@ def main():
         dist.barrier()
     launches = ctx.launch_count() - launches0
     total_ms = sum(a.elapsed_time(b) for a, b in evs)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=devn)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
-    value = world * args.steps / (max_ms / 1000.0)
+    max_ms = max_over_ranks(total_ms, world, devn)
+    value = job_value(world, args.steps, max_ms)
 
     # ---- per-kernel breakdown: the same steps again with the library's per-launch events (the
     # events add gaps between launches, so this pass is not part of `value`)
@@ -518,14 +539,11 @@ def main():
             b.record(stream)
             ev2.append((a, b))
         torch.cuda.synchronize()
-        e2e_ms = torch.tensor([sum(a.elapsed_time(b) for a, b in ev2)], dtype=torch.float64,
-                              device=devn)
-        if world > 1:
-            dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+        e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2), world, devn)
         bi = sum(x.numel() * x.element_size() for x in (h_pos, h_types, h_rp, h_ci)) + \
             (h_gp.numel() * 4 if G > 1 else 0)
         bo = h_energy.numel() * 4 + h_forces.numel() * 4
-        e2e = {"value": world * args.steps / (float(e2e_ms.item()) / 1000.0), "unit": UNIT,
+        e2e = {"value": job_value(world, args.steps, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo)}
     ck = clocks.stop() if clocks else None
     ctx.status_sync()
