@@ -217,18 +217,34 @@ extern "C" int mp_md_run(mp_ctx* c, int N, float* pos, float* vel, float* forces
   int builds = 0;
   StepGraph sg;
   // the list at the current positions, the reference positions, and energy/forces with it
+  // The forces at the current positions came from the old list; they are those of an exact r_c
+  // list as long as no atom has moved skin / 2 since that list was built (a pair now within r_c
+  // was then within r_c + skin). Only otherwise are they evaluated again with the new list.
+  const float half_skin = 0.5f * skin * 0.999f;
   auto build = [&]() -> int {
+    bool fresh_forces = builds == 0;
+    if (!fresh_forces) {  // read back by the synchronisation inside the list build
+      cudaMemsetAsync(c->md_flag, 0, sizeof(int), s);
+      int rc0 = launch(c, K_MD, k_displaced, dim3((N + 255) / 256), dim3(256), 0, s, N,
+                       (const float*)pos, (const float*)c->md_ref, half_skin * half_skin,
+                       c->md_flag);
+      if (rc0 != MP_OK) return rc0;
+      cudaMemcpyAsync(c->md_flag_h, c->md_flag, sizeof(int), cudaMemcpyDeviceToHost, s);
+    }
     int rc = mp_neighbor_csr(N, pos, graph_ptr, n_graphs, r_list, row_ptr, col_idx, capacity, &E,
                              stream);
     *n_edges = E;
     if (rc != MP_OK) return rc;
     if (E > c->cfg.max_edges) return MP_ERR_CAPACITY;
     ++builds;
+    if (!fresh_forces && *c->md_flag_h != 0) fresh_forces = true;
     if (N > 0 && cudaMemcpyAsync(c->md_ref, pos, sizeof(float) * 3 * (size_t)N,
                                  cudaMemcpyDeviceToDevice, s) != cudaSuccess)
       return MP_ERR_CUDA;
-    rc = energy_forces_launches(c, N, E, pos, types, row_ptr, col_idx, graph_ptr, n_graphs,
-                                energy, forces, s);
+    if (fresh_forces) {
+      rc = energy_forces_launches(c, N, E, pos, types, row_ptr, col_idx, graph_ptr, n_graphs,
+                                  energy, forces, s);
+    }
     if (rc == MP_OK && N > 0)
       record_step(c, sg, N, E, pos, vel, forces, inv_mass, dt, types, row_ptr, col_idx,
                   graph_ptr, n_graphs, energy, s);

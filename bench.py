@@ -446,7 +446,8 @@ def main():
     if not args.profile_run and rank == 0:
         skin, md_steps, dt = 0.5, 50, 0.005
         rp_s, ci_s = mp.neighbor_csr(pos_d, wl.r_c + skin, graph_ptr=gp_d)
-        ctx_md = mp.Context.from_workload(wl, weights, max_atoms=N, max_edges=ci_s.numel(),
+        # capacity for lists rebuilt later (atoms move; a list may grow a little)
+        ctx_md = mp.Context.from_workload(wl, weights, max_atoms=N, max_edges=2 * ci_s.numel(),
                                           max_graphs=G)
         im_d = (1.0 / (1.0 + types_d.float())).contiguous()
         vel = (torch.randn((N, 3), generator=torch.Generator(device=devn).manual_seed(7),

@@ -266,10 +266,12 @@ int mp_md_verlet(mp_ctx* ctx, int N, long long E, float* pos, float* vel, float*
  * check, once an atom has moved more than a displacement limit]. The call builds the list with
  * cutoff r_c + skin at the current positions (mp_neighbor_csr into row_ptr / col_idx, capacity
  * entries), evaluates energy and forces with it (`forces` need not hold anything on entry), then
- * runs n_steps steps of mp_md_verlet's scheme. It rebuilds the list, and re-evaluates energy and
- * forces at the current positions with the new list, after every rebuild_every steps (0: never
- * on a schedule) and after any check that finds an atom more than max_disp from where it was at
- * the last build (checked every check_every >= 1 steps; max_disp <= 0 disables it).
+ * runs n_steps steps of mp_md_verlet's scheme. It rebuilds the list after every rebuild_every
+ * steps (0: never on a schedule) and after any check that finds an atom more than max_disp from
+ * where it was at the last build (checked every check_every >= 1 steps; max_disp <= 0 disables
+ * it). At a rebuild the energy and forces of the current positions are evaluated again with the
+ * new list only if some atom has moved more than skin / 2 since the previous build (otherwise
+ * the old list already held every pair within r_c and they are unchanged).
  * The forces equal those of an exact r_c list at every step as long as no atom gets further than
  * skin / 2 from its position at the last build between two checks; max_disp <= skin / 2 with
  * check_every = 1 guarantees it.
