@@ -16,6 +16,7 @@
 #include <cmath>
 
 #include "mp_internal.cuh"
+#include "tc_api.cuh"
 
 namespace mp {
 namespace {
@@ -491,10 +492,13 @@ int run_attn_bwd(mp_ctx* c, int N, int K, const float* pos, const int* nbr,
   const int grid_d = (int)(N < cap_d ? N : cap_d), grid_s = (int)(N < cap_s ? N : cap_s);
   float* gq = c->g_x;     // [N][F] scratch: dL/dq
   float* gk = c->grad_h;  // [N][F] scratch: dL/dk
-  int rc = launch(c, K_ATTN_BWD, kd, dim3(grid_d), dim3(F), smem_dst, s, N, K, pos, nbr, mask,
-                  (const T*)x, g, (const float*)c->q, (const float*)c->k, filter_of(c, 0),
-                  radial_of(c), (const float*)c->P, (const float*)c->p, H, D, gq, grad_pos,
-                  c->attn_stats, c->status_d);
+  // destination pass: on the tensor cores where the bf16 kernel covers the shape
+  int rc = tc_attn_bwd_supported(c, K)
+               ? tc_attn_bwd_dst(c, N, K, pos, nbr, mask, x, g, gq, grad_pos, s)
+               : launch(c, K_ATTN_BWD, kd, dim3(grid_d), dim3(F), smem_dst, s, N, K, pos, nbr,
+                        mask, (const T*)x, g, (const float*)c->q, (const float*)c->k,
+                        filter_of(c, 0), radial_of(c), (const float*)c->P, (const float*)c->p, H,
+                        D, gq, grad_pos, c->attn_stats, c->status_d);
   if (rc == MP_OK)
     rc = launch(c, K_ATTN_BWD_SRC, ks, dim3(grid_s), dim3(F), 0, s, N, K, pos, rev_ptr, rev,
                 (const T*)x, g, (const float*)c->q, (const float*)c->k, filter_of(c, 0),

@@ -37,6 +37,12 @@ int tc_cfconv_bwd(mp_ctx* ctx, int block, int N, long long E, const float* pos, 
 bool tc_attn_supported(const mp_ctx* ctx, int K);
 int tc_attn_fwd(mp_ctx* ctx, int N, int K, const float* pos, const int* nbr,
                 const unsigned char* mask, const void* x, void* out, cudaStream_t s);
+// Destination pass of the attention backward on the tensor cores (tc_attn_bwd.cu): writes dL/dq
+// (scaled) into gq, the row side of dL/dr into grad_pos, and the rows' softmax statistics.
+bool tc_attn_bwd_supported(const mp_ctx* ctx, int K);
+int tc_attn_bwd_dst(mp_ctx* ctx, int N, int K, const float* pos, const int* nbr,
+                    const unsigned char* mask, const void* x, const float* g, float* gq,
+                    float* grad_pos, cudaStream_t s);
 // Atomwise layer on the tensor cores: out = in . W + b over rows (see tc_dense.cu for the modes).
 enum { TC_DENSE_STORE = 0, TC_DENSE_RESIDUAL = 1, TC_DENSE_READOUT = 2 };
 size_t tc_dense_bytes(int n_blocks);
