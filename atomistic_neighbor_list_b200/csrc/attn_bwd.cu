@@ -499,7 +499,9 @@ int run_attn_bwd(mp_ctx* c, int N, int K, const float* pos, const int* nbr,
                         mask, (const T*)x, g, (const float*)c->q, (const float*)c->k,
                         filter_of(c, 0), radial_of(c), (const float*)c->P, (const float*)c->p, H,
                         D, gq, grad_pos, c->attn_stats, c->status_d);
-  if (rc == MP_OK)
+  if (rc == MP_OK && tc_attn_bwd_supported(c, K))
+    rc = tc_attn_bwd_src(c, N, K, pos, rev_ptr, rev, x, g, grad_x, gk, grad_pos, s);
+  else if (rc == MP_OK)
     rc = launch(c, K_ATTN_BWD_SRC, ks, dim3(grid_s), dim3(F), 0, s, N, K, pos, rev_ptr, rev,
                 (const T*)x, g, (const float*)c->q, (const float*)c->k, filter_of(c, 0),
                 radial_of(c), (const float*)c->P, (const float*)c->p, H, D,

@@ -15,7 +15,8 @@ const char* kernel_name(int id) {
       "embed", "dense", "readout_energy", "readout_bwd", "graph_energy_sum", "cfconv_fwd_simt",
       "cfconv_bwd_simt", "attn_simt", "validate_csr", "cfconv_fwd_tc", "cfconv_bwd_tc",
       "attn_tc", "dense_tc", "md_integrate", "attn_bwd_dst", "attn_bwd_src",
-      "attn_transpose", "attn_eq_simt", "attn_bwd_dst_tc"};
+      "attn_transpose", "attn_eq_simt", "attn_bwd_dst_tc",
+      "attn_bwd_src_tc"};
   return (id >= 0 && id < K_NUM) ? names[id] : "?";
 }
 

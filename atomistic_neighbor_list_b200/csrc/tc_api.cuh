@@ -43,6 +43,11 @@ bool tc_attn_bwd_supported(const mp_ctx* ctx, int K);
 int tc_attn_bwd_dst(mp_ctx* ctx, int N, int K, const float* pos, const int* nbr,
                     const unsigned char* mask, const void* x, const float* g, float* gq,
                     float* grad_pos, cudaStream_t s);
+// Its source pass (needs the destination pass's statistics): writes the value path of dL/dx
+// into grad_x, dL/dk into gk, and adds the source side of dL/dr to grad_pos.
+int tc_attn_bwd_src(mp_ctx* ctx, int N, int K, const float* pos, const int* rev_ptr,
+                    const int* rev, const void* x, const float* g, float* grad_x, float* gk,
+                    float* grad_pos, cudaStream_t s);
 // Atomwise layer on the tensor cores: out = in . W + b over rows (see tc_dense.cu for the modes).
 enum { TC_DENSE_STORE = 0, TC_DENSE_RESIDUAL = 1, TC_DENSE_READOUT = 2 };
 size_t tc_dense_bytes(int n_blocks);

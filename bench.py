@@ -416,7 +416,8 @@ def main():
         ctx4.status_sync()
         msb = sum(a.elapsed_time(b) for a, b in evb) / len(evb)
         attn["backward"] = {"value": valid4 / (msb / 1000.0), "unit": "edges/s",
-                            "ms_per_call": msb, "path": "SIMT fp32 math, two passes"}
+                            "ms_per_call": msb,
+                            "path": "tcgen05 filter MMAs in both passes (bf16, K a multiple of 128)"}
         del g4, gx4, gp4
         # the equivariant value path (solid harmonics l <= 2 on each value), same timing rules
         oe4 = torch.empty((n4, 9, wl4.F), dtype=x4.dtype, device=devn)

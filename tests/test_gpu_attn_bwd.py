@@ -62,20 +62,21 @@ def test_attn_bwd_matches_oracle(mp, n, K, r_c, dtype):
 
 
 @pytest.mark.parametrize("n,K", [(2000, 128), (1500, 256)])
-def test_attn_bwd_tensor_core_destination_pass(mp, n, K):
-    """bf16, 16 heads x 8, K a multiple of 128: the destination pass runs on the tensor cores
-    (filter and its d-derivative from bf16 MMAs), so the bound is the bf16 one: dL/dx normwise
-    2e-2 (features), dL/dr relative RMS 1e-2 (forces)."""
+def test_attn_bwd_tensor_core_passes(mp, n, K):
+    """bf16, 16 heads x 8, K a multiple of 128: both passes run on the tensor cores (filter and
+    its d-derivative from bf16 MMAs, the source-side sums as MMAs of bf16 messages), so the bound
+    is the bf16 one: dL/dx normwise 2e-2 (features), dL/dr relative RMS 1e-2 (forces)."""
     wl, pos, nbr, mask, onbr, omask, ctx, x_t, x_ref, g, model = case(mp, n, K, 8.5, "bf16", 3)
     ctx.profile_begin()
     gx, gp = ctx.attn_bwd(dev(pos), nbr, mask, x_t.to(DEV), dev(g))
     prof = ctx.profile_end()
     ctx.status_sync()
-    assert "attn_bwd_dst_tc" in prof and "attn_bwd_dst" not in prof, prof
+    assert "attn_bwd_dst_tc" in prof and "attn_bwd_src_tc" in prof, prof
+    assert "attn_bwd_dst" not in prof and "attn_bwd_src" not in prof, prof
     rgx, rgp = oracle.attention_vjp(model, pos, onbr, omask, x_ref, g.astype(np.float64))
     ex = normwise(gx.cpu().numpy(), rgx)
     ep = rel_rms(gp.cpu().numpy(), rgp)
-    print(f"tc dst pass: grad_x normwise {ex:.2e}, grad_pos rel-rms {ep:.2e}")
+    print(f"tc passes: grad_x normwise {ex:.2e}, grad_pos rel-rms {ep:.2e}")
     assert ex <= TOL_BF16_FEAT and ep <= TOL_BF16_FORCE, (ex, ep)
 
 
@@ -122,5 +123,5 @@ def test_attn_bwd_full_size_sampled(mp):
         errs.append((np.abs(gx[k] - rgx[k]).max() / np.abs(rgx[k]).max(),
                      np.linalg.norm(gp[k] - rgp[k]) / np.linalg.norm(rgp[k])))
     print("sampled atoms (grad_x, grad_pos) relative errors", errs)
-    # bf16 tensor-core destination pass: per-atom bounds at twice the bf16 feature / force bounds
+    # bf16 tensor-core passes: per-atom bounds at twice the bf16 feature / force bounds
     assert all(a <= 2 * TOL_BF16_FEAT and b <= 2 * TOL_BF16_FORCE for a, b in errs), errs
