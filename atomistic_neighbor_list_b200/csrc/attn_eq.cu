@@ -9,30 +9,13 @@
 // edge on chip from the edge vector the distance already needs -- the same sum, streamed, with no
 // edge tensor in memory and one online softmax (running maximum and normaliser) per head.
 #include "mp_internal.cuh"
+#include "tc_api.cuh"
 
 namespace mp {
 namespace {
 
 constexpr int QB = 16;  // slots per batch
 constexpr int NSH = 9;  // solid harmonics l <= 2
-
-// the nine solid harmonics of (x, y, z), in the order (0,0), (1,-1), (1,0), (1,1), (2,-2), ...
-__device__ __forceinline__ void solid_harmonics9(float x, float y, float z, float* S) {
-  const float c0 = 0.28209479177387814f;   // 1 / (2 sqrt(pi))
-  const float c1 = 0.48860251190291992f;   // sqrt(3 / (4 pi))
-  const float c2 = 1.09254843059207907f;   // sqrt(15 / pi) / 2
-  const float c20 = 0.31539156525252005f;  // sqrt(5 / pi) / 4
-  const float c22 = 0.54627421529603953f;  // sqrt(15 / pi) / 4
-  S[0] = c0;
-  S[1] = c1 * y;
-  S[2] = c1 * z;
-  S[3] = c1 * x;
-  S[4] = c2 * x * y;
-  S[5] = c2 * y * z;
-  S[6] = c20 * (2.f * z * z - x * x - y * y);
-  S[7] = c2 * x * z;
-  S[8] = c22 * (x * x - y * y);
-}
 
 template <typename T, int F>
 __global__ void __launch_bounds__(F) k_attn_eq_simt(
@@ -179,6 +162,7 @@ extern "C" int mp_attn_eq_fwd(mp_ctx* c, int N, int K, const float* pos, const i
   int rc = launch_dense(c, N, F, F, x, bf, c->Wq, nullptr, false, c->q, false, s);
   if (rc == MP_OK) rc = launch_dense(c, N, F, F, x, bf, c->Wk, nullptr, false, c->k, false, s);
   if (rc != MP_OK) return rc;
+  if (tc_attn_eq_supported(c, K)) return tc_attn_eq_fwd(c, N, K, pos, nbr, mask, x, out, s);
   if (F == 64)
     return bf ? run_attn_eq<__nv_bfloat16, 64>(c, N, K, pos, nbr, mask, x, out, s)
               : run_attn_eq<float, 64>(c, N, K, pos, nbr, mask, x, out, s);

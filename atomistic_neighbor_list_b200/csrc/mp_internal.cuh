@@ -35,7 +35,7 @@ enum KernelId : int {
   K_EMBED = 0, K_DENSE, K_READOUT_E, K_READOUT_BWD, K_GRAPH_SUM, K_CFCONV_FWD_SIMT,
   K_CFCONV_BWD_SIMT, K_ATTN_SIMT, K_VALIDATE, K_CFCONV_FWD_TC, K_CFCONV_BWD_TC, K_ATTN_TC,
   K_DENSE_TC, K_MD, K_ATTN_BWD, K_ATTN_BWD_SRC, K_ATTN_REV, K_ATTN_EQ,
-  K_ATTN_BWD_TC, K_ATTN_BWD_SRC_TC, K_NUM
+  K_ATTN_BWD_TC, K_ATTN_BWD_SRC_TC, K_ATTN_EQ_TC, K_NUM
 };
 const char* kernel_name(int id);
 
@@ -151,6 +151,26 @@ __device__ __forceinline__ float cutoff_f(float d, float rc) {
 }
 __device__ __forceinline__ float cutoff_grad_f(float d, float rc) {
   return d < rc ? -0.5f * 3.14159265358979f / rc * sinpif(d / rc) : 0.f;
+}
+
+// The nine regular solid harmonics |r|^l Y_lm(r/|r|), l <= 2, of r = (x, y, z), Y the real
+// spherical harmonics orthonormal on the sphere, in the order (0,0), (1,-1), (1,0), (1,1), (2,-2),
+// (2,-1), (2,0), (2,1), (2,2) (E2Former-V2 page s.3.1: the geometry of the value path).
+__device__ __forceinline__ void solid_harmonics9(float x, float y, float z, float* S) {
+  const float c0 = 0.28209479177387814f;   // 1 / (2 sqrt(pi))
+  const float c1 = 0.48860251190291992f;   // sqrt(3 / (4 pi))
+  const float c2 = 1.09254843059207907f;   // sqrt(15 / pi) / 2
+  const float c20 = 0.31539156525252005f;  // sqrt(5 / pi) / 4
+  const float c22 = 0.54627421529603953f;  // sqrt(15 / pi) / 4
+  S[0] = c0;
+  S[1] = c1 * y;
+  S[2] = c1 * z;
+  S[3] = c1 * x;
+  S[4] = c2 * x * y;
+  S[5] = c2 * y * z;
+  S[6] = c20 * (2.f * z * z - x * x - y * y);
+  S[7] = c2 * x * z;
+  S[8] = c22 * (x * x - y * y);
 }
 
 __device__ __forceinline__ void raise_status(int* status, int bit) {

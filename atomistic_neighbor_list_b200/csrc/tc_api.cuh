@@ -37,6 +37,11 @@ int tc_cfconv_bwd(mp_ctx* ctx, int block, int N, long long E, const float* pos, 
 bool tc_attn_supported(const mp_ctx* ctx, int K);
 int tc_attn_fwd(mp_ctx* ctx, int N, int K, const float* pos, const int* nbr,
                 const unsigned char* mask, const void* x, void* out, cudaStream_t s);
+// The attention with the equivariant value path (9 solid harmonics, out [N][9][F]) on the same
+// tensor-core kernel, one weighted-sum MMA per harmonic (tc_attn.cu).
+bool tc_attn_eq_supported(const mp_ctx* ctx, int K);
+int tc_attn_eq_fwd(mp_ctx* ctx, int N, int K, const float* pos, const int* nbr,
+                   const unsigned char* mask, const void* x, void* out, cudaStream_t s);
 // Destination pass of the attention backward on the tensor cores (tc_attn_bwd.cu): writes dL/dq
 // (scaled) into gq, the row side of dL/dr into grad_pos, and the rows' softmax statistics.
 bool tc_attn_bwd_supported(const mp_ctx* ctx, int K);

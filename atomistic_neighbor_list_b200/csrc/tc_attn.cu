@@ -52,7 +52,7 @@ struct AtRed {  // per-tile softmax partials (double-buffered)
 struct AtSmem {
   uint32_t w1, w2, c2, a0, p, h0, x, meta0, red0, misc, bars, total;
 };
-__host__ __device__ constexpr AtSmem at_layout(int K1) {
+__host__ __device__ constexpr AtSmem at_layout(int K1, int NC) {
   // W1 | P (144 rows) | W2 | c2 | Gaussian operand x2 | p operand | h' / v^T x2 | x_j rows |
   // metadata x4 | softmax partials x2 | misc | mbarriers
   AtSmem L{};
@@ -61,7 +61,7 @@ __host__ __device__ constexpr AtSmem at_layout(int K1) {
   L.w2 = o;    o += FT * K2 * 2;
   L.c2 = o;    o += 1024;
   L.a0 = o;    o += 2 * TM * K1 * 2;
-  L.p = o;     o += AH * TM * 2;
+  L.p = o;     o += AH * TM * 2 * NC;
   L.h0 = o;    o += 2 * TM * K2 * 2;
   L.x = o;     o += TM * FT * 2;
   L.meta0 = o; o += NMETA * (uint32_t)sizeof(AtMeta);
@@ -71,7 +71,9 @@ __host__ __device__ constexpr AtSmem at_layout(int K1) {
   L.total = o;
   return L;
 }
-__host__ __device__ constexpr bool at_fits(int K1) { return at_layout(K1).total + 1024 <= 227 * 1024; }
+__host__ __device__ constexpr bool at_fits(int K1, int NC) {
+  return at_layout(K1, NC).total + 1024 <= 227 * 1024;
+}
 __device__ __forceinline__ uint32_t xoff(int r, int c) {  // staged x_j rows (bank-permuted)
   return (uint32_t)(r * (FT * 2) + ((c ^ (r & 7)) << 4));
 }
@@ -83,7 +85,10 @@ enum {
   N_BARS = 28
 };
 
-template <int K1>
+// NC = 1: the attention of the scalar values; NC = 9: each value also coupled with the solid
+// harmonics l <= 2 of r_j - r_i (one weighted-sum MMA per harmonic, p scaled by S_lm(r_ij)), out
+// [N][9][F] (E2Former-V2 page s.3.1: direction only through the value path).
+template <int K1, int NC>
 __global__ void __launch_bounds__(AT_THREADS, 1) k_attn_tc(
     int N, int K, const float* __restrict__ pos, const int* __restrict__ nbr,
     const unsigned char* __restrict__ mask, const __nv_bfloat16* __restrict__ x,
@@ -92,7 +97,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1) k_attn_tc(
     int* status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  constexpr AtSmem L = at_layout(K1);
+  constexpr AtSmem L = at_layout(K1, NC);
   uint8_t* sW1 = sm + L.w1;  // rows 0..127 W1 (bias c1 on column R), rows 128..143 P (bias p)
   uint8_t* sW2 = sm + L.w2;
   float* sc2 = (float*)(sm + L.c2);
@@ -289,10 +294,11 @@ __global__ void __launch_bounds__(AT_THREADS, 1) k_attn_tc(
         if (!(ok = wait_bar(B_FULL_M + b, par))) break;
         tc::fence_after();
         // D^T[F x 16 heads] = v^T (MN-major) . p^T (K-major): each feature's own head column is
-        // the tile's softmax-weighted sum for it
-        for (int ks = 0; ks < TM / 16; ++ks)
-          tc::mma(tmem + 256 * b, tc::sdesc(sH_a + ks * 256, 128, 2048),
-                  tc::sdesc(sP_a + ks * 256, 128, TM * 16), id3, ks > 0);
+        // the tile's softmax-weighted sum for it; one such product per harmonic
+        for (int m = 0; m < NC; ++m)
+          for (int ks = 0; ks < TM / 16; ++ks)
+            tc::mma(tmem + 256 * b + 16 * m, tc::sdesc(sH_a + ks * 256, 128, 2048),
+                    tc::sdesc(sP_a + m * (AH * TM * 2) + ks * 256, 128, TM * 16), id3, ks > 0);
         tc::commit(&bars[B_DONE3 + b]);
       }
       if (!ok) *abort_flag = 1;
@@ -307,7 +313,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1) k_attn_tc(
     const int e_me = 32 * q4 + lane;          // slot = TMEM lane (drain: feature)
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q4) << 16);
     float bias[4] = {0.f, 0.f, 0.f, 0.f};     // this slot's radial logit bias, E1(i) -> E2(i)
-    float m_run = -INFINITY, z_run = 0.f, acc_run = 0.f;  // drain: the atom's running softmax
+    float m_run = -INFINITY, z_run = 0.f, acc_run[NC];    // drain: the atom's running softmax
+#pragma unroll
+    for (int m = 0; m < NC; ++m) acc_run[m] = 0.f;
     auto arrive_warp = [&](int idx) {
       tc::fence_proxy_async();
       tc::fence_before();
@@ -409,9 +417,24 @@ __global__ void __launch_bounds__(AT_THREADS, 1) k_attn_tc(
       tc::fence_after();
       // the p operand has one buffer: MMA3 of tile i-1 was issued before MMA2 of tile i, whose
       // completion this warp just saw
+      if constexpr (NC == 1) {
 #pragma unroll
-      for (int hh = 0; hh < 4; ++hh)
-        *(__nv_bfloat16*)(sP + kmaj(h0 + hh, e_me, TM)) = __float2bfloat16_rn(pb[hh]);
+        for (int hh = 0; hh < 4; ++hh)
+          *(__nv_bfloat16*)(sP + kmaj(h0 + hh, e_me, TM)) = __float2bfloat16_rn(pb[hh]);
+      } else {  // one operand per harmonic: p S_lm(r_j - r_i) (p is 0 on a padded slot)
+        float S[9] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (ok) {
+          const int j = M->src[e_me], a = M->atom;
+          solid_harmonics9(pos[3 * j] - pos[3 * a], pos[3 * j + 1] - pos[3 * a + 1],
+                           pos[3 * j + 2] - pos[3 * a + 2], S);
+        }
+#pragma unroll
+        for (int m = 0; m < NC; ++m)
+#pragma unroll
+          for (int hh = 0; hh < 4; ++hh)
+            *(__nv_bfloat16*)(sP + m * (AH * TM * 2) + kmaj(h0 + hh, e_me, TM)) =
+                __float2bfloat16_rn(pb[hh] * S[m]);
+      }
       uint8_t* H = HB(b);
       uint32_t r[32];
       tc::ld32(lane_base + 256 * b + f0, r);
@@ -447,34 +470,47 @@ __global__ void __launch_bounds__(AT_THREADS, 1) k_attn_tc(
         tc::fence_after();
         const AtMeta* M = MB(i % NMETA);
         const AtRed* R = RB(b);
-        uint32_t v4[4];
-        tc::ld4(lane_base + 256 * b + 4 * q4, v4);  // heads 4 q4 .. 4 q4 + 3 of this warp's features
-        tc::ld_wait();
         const int hs = lane >> 3, hf = 4 * q4 + hs;
-        const float acc_t = __uint_as_float(hs == 0 ? v4[0] : hs == 1 ? v4[1] : hs == 2 ? v4[2] : v4[3]);
+        float acc_t[NC];
+#pragma unroll
+        for (int m = 0; m < NC; ++m) {  // heads 4 q4 .. 4 q4 + 3 of this warp's features
+          uint32_t v4[4];
+          tc::ld4(lane_base + 256 * b + 16 * m + 4 * q4, v4);
+          tc::ld_wait();
+          acc_t[m] = __uint_as_float(hs == 0 ? v4[0] : hs == 1 ? v4[1] : hs == 2 ? v4[2] : v4[3]);
+        }
         const float m_t = R->mh[hf];
         const float z_t = ((R->wsum[hf >> 2][0][hf & 3] + R->wsum[hf >> 2][1][hf & 3]) +
                            R->wsum[hf >> 2][2][hf & 3]) + R->wsum[hf >> 2][3][hf & 3];
         if (M->first) {
           m_run = -INFINITY;
           z_run = 0.f;
-          acc_run = 0.f;
+#pragma unroll
+          for (int m = 0; m < NC; ++m) acc_run[m] = 0.f;
         }
         if (m_t != -INFINITY) {  // a tile with no valid slot adds nothing
           if (m_run == -INFINITY) {
             m_run = m_t;
             z_run = z_t;
-            acc_run = acc_t;
+#pragma unroll
+            for (int m = 0; m < NC; ++m) acc_run[m] = acc_t[m];
           } else {
             const float mn = fmaxf(m_run, m_t);
             const float s1 = tc::ex2f((m_run - mn) * LOG2E), s2 = tc::ex2f((m_t - mn) * LOG2E);
-            acc_run = fmaf(acc_run, s1, acc_t * s2);
+#pragma unroll
+            for (int m = 0; m < NC; ++m) acc_run[m] = fmaf(acc_run[m], s1, acc_t[m] * s2);
             z_run = fmaf(z_run, s1, z_t * s2);
             m_run = mn;
           }
         }
-        if (M->last)
-          out[(size_t)M->atom * FT + e_me] = __float2bfloat16_rn(z_run > 0.f ? acc_run / z_run : 0.f);
+        if (M->last) {
+          const float iz = z_run > 0.f ? 1.f / z_run : 0.f;
+#pragma unroll
+          for (int m = 0; m < NC; ++m)
+            out[((size_t)M->atom * NC + m) * FT + e_me] =
+                __float2bfloat16_rn(NC == 1 ? (z_run > 0.f ? acc_run[m] / z_run : 0.f)
+                                            : acc_run[m] * iz);
+        }
       }
       tc::fence_before();
       __syncwarp();
@@ -501,28 +537,43 @@ __global__ void __launch_bounds__(AT_THREADS, 1) k_attn_tc(
 bool tc_attn_supported(const mp_ctx* ctx, int K) {
   const mp_config& c = ctx->cfg;
   return tc_supported(ctx) && ctx->tc_attn_p && c.n_heads == AH && c.head_dim == AD &&
-         K % TM == 0 && at_fits(k1_of(c.n_rbf));
+         K % TM == 0 && at_fits(k1_of(c.n_rbf), 1);
 }
 
-int tc_attn_fwd(mp_ctx* ctx, int N, int K, const float* pos, const int* nbr,
-                const unsigned char* mask, const void* x, void* out, cudaStream_t s) {
+template <int NC>
+int tc_attn_launch(mp_ctx* ctx, int N, int K, const float* pos, const int* nbr,
+                   const unsigned char* mask, const void* x, void* out, cudaStream_t s) {
   const int K1 = k1_of(ctx->cfg.n_rbf);
   const uint8_t* img = (const uint8_t*)ctx->tc_weights;  // the filter of block 0
   int grid = ctx->num_sms;
   if (N < grid) grid = N > 0 ? N : 1;
   const float qscale = 1.f / sqrtf((float)AD);
   auto go = [&](auto kern, int k1) {
-    const size_t smem = at_layout(k1).total + 1024;
+    const size_t smem = at_layout(k1, NC).total + 1024;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    return launch(ctx, K_ATTN_TC, kern, dim3(grid), dim3(AT_THREADS), smem, s, N, K, pos, nbr, mask,
-                  (const __nv_bfloat16*)x, (const float*)ctx->q, (const float*)ctx->k,
-                  (__nv_bfloat16*)out, img, (const uint8_t*)ctx->tc_attn_p, radial_of(ctx), qscale,
-                  ctx->status_d);
+    return launch(ctx, NC == 1 ? K_ATTN_TC : K_ATTN_EQ_TC, kern, dim3(grid), dim3(AT_THREADS),
+                  smem, s, N, K, pos, nbr, mask, (const __nv_bfloat16*)x, (const float*)ctx->q,
+                  (const float*)ctx->k, (__nv_bfloat16*)out, img, (const uint8_t*)ctx->tc_attn_p,
+                  radial_of(ctx), qscale, ctx->status_d);
   };
-  if (K1 == 64) return go(k_attn_tc<64>, 64);
-  if (K1 == 48) return go(k_attn_tc<48>, 48);
-  if (K1 == 32) return go(k_attn_tc<32>, 32);
+  if (K1 == 64) return go(k_attn_tc<64, NC>, 64);
+  if (K1 == 48) return go(k_attn_tc<48, NC>, 48);
+  if (K1 == 32) return go(k_attn_tc<32, NC>, 32);
   return MP_ERR_INVALID_ARG;
+}
+
+int tc_attn_fwd(mp_ctx* ctx, int N, int K, const float* pos, const int* nbr,
+                const unsigned char* mask, const void* x, void* out, cudaStream_t s) {
+  return tc_attn_launch<1>(ctx, N, K, pos, nbr, mask, x, out, s);
+}
+
+bool tc_attn_eq_supported(const mp_ctx* ctx, int K) {
+  return tc_attn_supported(ctx, K) && at_fits(k1_of(ctx->cfg.n_rbf), 9);
+}
+
+int tc_attn_eq_fwd(mp_ctx* ctx, int N, int K, const float* pos, const int* nbr,
+                   const unsigned char* mask, const void* x, void* out, cudaStream_t s) {
+  return tc_attn_launch<9>(ctx, N, K, pos, nbr, mask, x, out, s);
 }
 
 }  // namespace mp

@@ -434,7 +434,8 @@ def main():
         ctx4.status_sync()
         mse = sum(a.elapsed_time(b) for a, b in eve) / len(eve)
         attn["equivariant"] = {"value": valid4 / (mse / 1000.0), "unit": "edges/s",
-                               "ms_per_call": mse, "path": "SIMT fp32 math, l <= 2"}
+                               "ms_per_call": mse,
+                               "path": "tcgen05: one weighted-sum MMA per harmonic, l <= 2"}
         del oe4
         ctx4.close()
         del nbr4, mask4, x4, o4, pos4_d

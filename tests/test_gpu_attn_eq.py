@@ -70,3 +70,27 @@ def test_attn_eq_full_size_sampled(mp):
     ref = oracle.attention_equivariant(model, pos, onbr, omask, x_ref, rows=rows)
     for lo, hi in ((0, 1), (1, 4), (4, 9)):
         assert normwise(got[rows, lo:hi], ref[:, lo:hi]) <= TOL_BF16_FEAT, (lo, hi)
+
+
+@pytest.mark.parametrize("n,K", [(2000, 128), (1500, 256)])
+def test_attn_eq_tensor_core_path(mp, n, K):
+    """bf16, 16 heads x 8, K a multiple of 128: the tensor-core kernel (one weighted-sum MMA per
+    harmonic, p S_lm as bf16 operands); each l block within the bf16 feature bound."""
+    wl = dataclasses.replace(synth.WORKLOADS["cfg4"], n_atoms=n, K=K)
+    pos = synth.uniform_positions(n, seed=2)
+    w = synth.make_weights(wl)
+    nbr, mask = mp.neighbor_padded(dev(pos), wl.r_c, K)
+    onbr, omask = oracle_padded(pos, wl.r_c, K, nbr, mask)
+    ctx = mp.Context.from_workload(wl, w, max_atoms=n, max_edges=1)
+    x_t, x_ref = features_for(synth.node_features(n, wl.F, seed=5), "bf16")
+    ctx.profile_begin()
+    out = ctx.attn_eq_fwd(dev(pos), nbr, mask, x_t.to(DEV))
+    prof = ctx.profile_end()
+    ctx.status_sync()
+    assert "attn_eq_tc" in prof and "attn_eq_simt" not in prof, prof
+    model = oracle.Model.from_workload(wl, oracle_weights(w, "bf16"))
+    ref = oracle.attention_equivariant(model, pos, onbr, omask, x_ref)
+    got = out.float().cpu().numpy().astype(np.float64)
+    errs = [normwise(got[:, lo:hi], ref[:, lo:hi]) for lo, hi in ((0, 1), (1, 4), (4, 9))]
+    print("tc equivariant attention, per l block:", errs)
+    assert max(errs) <= TOL_BF16_FEAT, errs
