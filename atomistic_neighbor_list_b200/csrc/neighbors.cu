@@ -377,9 +377,44 @@ __global__ void __launch_bounds__(kFillWarps * 32) k_cell_fill(
   }
 }
 
+// Bitonic sorting network over P (a power of two) staged entries of one warp, ascending by
+// (d2, j) or by j alone; every lane takes P / 64 compare-exchanges per stage.
+__device__ __forceinline__ void warp_bitonic(int* __restrict__ sj, double* __restrict__ sd, int P,
+                                             bool by_dist) {
+  const int lane = threadIdx.x & 31;
+  for (int k = 2; k <= P; k <<= 1) {
+    for (int h = k >> 1; h > 0; h >>= 1) {
+      for (int i = lane; i < P; i += 32) {
+        const int l = i ^ h;
+        if (l > i) {
+          const int ji = sj[i], jl = sj[l];
+          bool gt;
+          if (by_dist) {
+            const double di = sd[i], dl = sd[l];
+            gt = di > dl || (di == dl && ji > jl);
+          } else {
+            gt = ji > jl;
+          }
+          if (gt == ((i & k) == 0)) {  // out of order for this block's direction
+            sj[i] = jl;
+            sj[l] = ji;
+            if (by_dist) {
+              const double t = sd[i];
+              sd[i] = sd[l];
+              sd[l] = t;
+            }
+          }
+        }
+      }
+      __syncwarp();
+    }
+  }
+}
+
 // Padded list: the hits of a row staged as (j, d2); with more than K, keep those whose rank by
-// (d2, j) is below K; kept entries are written in ascending j. A row with more than 1024 hits
-// raises the overflow flag and is written empty.
+// (d2, j) is below K (a sorting network by (d2, j)); kept entries are written in ascending j (a
+// sorting network by j). A row with more than 1024 hits raises the overflow flag and is written
+// empty.
 constexpr int kPadCap = 1024, kPadWarps = 4;
 
 __global__ void __launch_bounds__(kPadWarps * 32) k_cell_padded(
@@ -427,31 +462,27 @@ __global__ void __launch_bounds__(kPadWarps * 32) k_cell_padded(
       if (lane == 0) *overflow = 1;
       n = 0;
     }
-    if (n > K) {  // drop all but the K nearest by (d2, j): a dropped entry's j becomes INT_MAX
-      unsigned drop = 0;
-      for (int c = lane, t = 0; c < n; c += 32, ++t) {
-        const int jc = sj[c];
-        const double dc = sd[c];
-        int r = 0;
-        for (int o = 0; o < n; ++o) {
-          const double dd = sd[o];
-          r += (dd < dc || (dd == dc && sj[o] < jc)) ? 1 : 0;
-        }
-        if (r >= K) drop |= 1u << t;
-      }
-      __syncwarp();
-      for (int c = lane, t = 0; c < n; c += 32, ++t)
-        if (drop >> t & 1u) sj[c] = 0x7fffffff;
-      __syncwarp();
+    // sorting network over the staged hits, padded to a power of two with entries that sort last
+    int P = 1;
+    while (P < n) P <<= 1;
+    for (int c = n + lane; c < P; c += 32) {
+      sj[c] = 0x7fffffff;
+      sd[c] = INFINITY;
     }
-    const int kept = n < K ? n : K;
-    for (int c = lane; c < n; c += 32) {  // kept entries at their rank by j
-      const int jc = sj[c];
-      if (jc == 0x7fffffff) continue;
-      int r = 0;
-      for (int o = 0; o < n; ++o) r += sj[o] < jc ? 1 : 0;
-      row_n[r] = jc;
-      row_m[r] = 1;
+    __syncwarp();
+    int kept = n;
+    if (n > K) {  // the K nearest by (d2, j) come first; the rest are dropped
+      warp_bitonic(sj, sd, P, true);
+      for (int c = K + lane; c < P; c += 32) sj[c] = 0x7fffffff;
+      __syncwarp();
+      kept = K;
+      P = 1;
+      while (P < K) P <<= 1;
+    }
+    warp_bitonic(sj, sd, P, false);  // the kept entries by ascending j
+    for (int c = lane; c < kept; c += 32) {
+      row_n[c] = sj[c];
+      row_m[c] = 1;
     }
     for (int s = kept + lane; s < K; s += 32) {
       row_n[s] = -1;
