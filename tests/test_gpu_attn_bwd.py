@@ -125,3 +125,21 @@ def test_attn_bwd_full_size_sampled(mp):
     print("sampled atoms (grad_x, grad_pos) relative errors", errs)
     # bf16 tensor-core passes: per-atom bounds at twice the bf16 feature / force bounds
     assert all(a <= 2 * TOL_BF16_FEAT and b <= 2 * TOL_BF16_FORCE for a, b in errs), errs
+
+
+def test_attn_bwd_tensor_core_empty_rows_and_determinism(mp):
+    """The tensor-core passes with rows that have no valid slot (their statistics are empty and
+    no source sees them) give the oracle's gradients, and the same bits twice."""
+    wl, pos, nbr, mask, onbr, omask, ctx, x_t, x_ref, g, model = case(mp, 1200, 128, 8.5, "bf16", 4)
+    omask = omask.copy()
+    omask[::5] = 0
+    omask[1::7, 64:] = 0  # some rows keep only their first tile
+    nbr, mask = dev(onbr), dev(omask)
+    a = ctx.attn_bwd(dev(pos), nbr, mask, x_t.to(DEV), dev(g))
+    b = ctx.attn_bwd(dev(pos), nbr, mask, x_t.to(DEV), dev(g))
+    torch.cuda.synchronize()
+    ctx.status_sync()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    rgx, rgp = oracle.attention_vjp(model, pos, onbr, omask, x_ref, g.astype(np.float64))
+    assert normwise(a[0].cpu().numpy(), rgx) <= TOL_BF16_FEAT
+    assert rel_rms(a[1].cpu().numpy(), rgp) <= TOL_BF16_FORCE

@@ -94,3 +94,24 @@ def test_attn_eq_tensor_core_path(mp, n, K):
     errs = [normwise(got[:, lo:hi], ref[:, lo:hi]) for lo, hi in ((0, 1), (1, 4), (4, 9))]
     print("tc equivariant attention, per l block:", errs)
     assert max(errs) <= TOL_BF16_FEAT, errs
+
+
+def test_attn_eq_tensor_core_empty_rows(mp):
+    wl = dataclasses.replace(synth.WORKLOADS["cfg4"], n_atoms=1000, K=128)
+    pos = synth.uniform_positions(1000, seed=6)
+    w = synth.make_weights(wl)
+    nbr, mask = mp.neighbor_padded(dev(pos), wl.r_c, 128)
+    onbr, omask = oracle_padded(pos, wl.r_c, 128, nbr, mask)
+    omask = omask.copy()
+    omask[::4] = 0
+    ctx = mp.Context.from_workload(wl, w, max_atoms=1000, max_edges=1)
+    x_t, x_ref = features_for(synth.node_features(1000, wl.F, seed=7), "bf16")
+    out = ctx.attn_eq_fwd(dev(pos), dev(onbr), dev(omask), x_t.to(DEV))
+    torch.cuda.synchronize()
+    ctx.status_sync()
+    got = out.float().cpu().numpy()
+    assert np.all(got[::4] == 0)  # no valid neighbor: zero rows
+    model = oracle.Model.from_workload(wl, oracle_weights(w, "bf16"))
+    ref = oracle.attention_equivariant(model, pos, onbr, omask, x_ref)
+    for lo, hi in ((0, 1), (1, 4), (4, 9)):
+        assert normwise(got[:, lo:hi], ref[:, lo:hi]) <= TOL_BF16_FEAT
