@@ -20,6 +20,8 @@ constexpr int BT = 256;          // threads
 constexpr int BH = 16, BD = 8;   // heads, head width
 constexpr int BN1 = FT + BH;     // MMA1 columns: the filter's first layer and the radial bias
 constexpr int KMAX = 256;        // slots per row this kernel keeps on chip
+constexpr int SLS = KMAX + 16;   // row stride of the per-head slot arrays (the two half warps of
+                                 // a statistics pass land on disjoint banks)
 
 struct BwSmem {
   uint32_t w1, w2, c2, x, row, total;
@@ -35,7 +37,7 @@ __host__ __device__ constexpr BwSmem bw_layout(int K1) {
   L.row = o;
   // per slot: logit, dalpha, beta, b' [16] each, unit vector [3], source; q_i, g_i; statistics;
   // per-tile geometry (fc, f_c', source) and reduction scratch
-  o += KMAX * (4 * BH + 4) * 4 + 2 * FT * 4 + 3 * BH * 4 + 3 * TM * 4 + 64 * 4;
+  o += (4 * BH * SLS + 4 * KMAX) * 4 + 2 * FT * 4 + 3 * BH * 4 + 3 * TM * 4 + 64 * 4;
   o += 64;  // mbarriers and the TMEM slot
   L.total = o;
   return L;
@@ -188,11 +190,11 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_dst_tc(
   uint8_t* sW2 = sm + L.w2;
   float* sc2 = (float*)(sm + L.c2);
   uint8_t* sX = sm + L.x;
-  float* s_l = (float*)(sm + L.row);         // [KMAX][16]
-  float* s_da = s_l + KMAX * BH;             // [KMAX][16]
-  float* s_be = s_da + KMAX * BH;            // [KMAX][16]
-  float* s_bp = s_be + KMAX * BH;            // [KMAX][16]
-  float* s_u = s_bp + KMAX * BH;             // [KMAX][3]
+  float* s_l = (float*)(sm + L.row);         // [16][SLS]: per head, per slot
+  float* s_da = s_l + BH * SLS;              // [16][SLS]
+  float* s_be = s_da + BH * SLS;             // [16][SLS]
+  float* s_bp = s_be + BH * SLS;             // [16][SLS]
+  float* s_u = s_bp + BH * SLS;              // [KMAX][3]
   int* s_src = (int*)(s_u + 3 * KMAX);       // [KMAX], -1: no valid neighbor in the slot
   float* s_q = (float*)(s_src + KMAX);       // [F], scaled by qscale
   float* s_g = s_q + FT;                     // [F]
@@ -311,7 +313,7 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_dst_tc(
             be = fmaf(gx, Wp, be);
           }
           if (ok) {
-            const int o = (s0 + e) * BH + 8 * half + hh;
+            const int o = (8 * half + hh) * SLS + s0 + e;
             s_l[o] = l + __uint_as_float(rb[hh]);
             s_da[o] = da;
             s_be[o] = be;
@@ -329,16 +331,16 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_dst_tc(
       const int h = tid >> 4, c = tid & 15;
       float m = -INFINITY;
       for (int s = c; s < K; s += 16)
-        if (s_src[s] >= 0) m = fmaxf(m, s_l[s * BH + h]);
+        if (s_src[s] >= 0) m = fmaxf(m, s_l[h * SLS + s]);
       for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
       float z = 0.f;
       for (int s = c; s < K; s += 16)
-        if (s_src[s] >= 0) z += tc::ex2f((s_l[s * BH + h] - m) * LOG2E);
+        if (s_src[s] >= 0) z += tc::ex2f((s_l[h * SLS + s] - m) * LOG2E);
       for (int o = 8; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
       const float iz = z > 0.f ? 1.f / z : 0.f;
       float D = 0.f;
       for (int s = c; s < K; s += 16)
-        if (s_src[s] >= 0) D += tc::ex2f((s_l[s * BH + h] - m) * LOG2E) * iz * s_da[s * BH + h];
+        if (s_src[s] >= 0) D += tc::ex2f((s_l[h * SLS + s] - m) * LOG2E) * iz * s_da[h * SLS + s];
       for (int o = 8; o > 0; o >>= 1) D += __shfl_xor_sync(0xffffffffu, D, o);
       if (c == 0) {
         s_st[h] = m;
@@ -367,7 +369,7 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_dst_tc(
         for (int u8 = 0; u8 < 8; ++u8) {
           const int s = s0 + 2 * u8;
           if (s < K && s_src[s] >= 0) {
-            const int o = s * BH + h;
+            const int o = h * SLS + s;
             const float a = tc::ex2f((s_l[o] - m) * LOG2E) * iz;
             acc = fmaf(a * (s_da[o] - D), kv[u8], acc);
           }
@@ -385,7 +387,7 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_dst_tc(
         if (s_src[s] < 0) continue;
         float sd = 0.f;
         for (int h = 0; h < BH; ++h) {
-          const int o = s * BH + h;
+          const int o = h * SLS + s;
           const float a = tc::ex2f((s_l[o] - s_st[h]) * LOG2E) * s_st[BH + h];
           sd = fmaf(a, s_be[o], sd);
           sd = fmaf(a * (s_da[o] - s_st[2 * BH + h]), s_bp[o], sd);
