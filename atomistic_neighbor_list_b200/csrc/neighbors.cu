@@ -253,7 +253,9 @@ __global__ void k_cell_assign(int N, const float* __restrict__ pos, const int* _
   const int id = cell_off[g] + (cz * cg.dim[1] + cy) * cg.dim[0] + cx;
   cellinfo[i] = make_int4(cx, cy, cz, g);
   cell_id[i] = id;
-  atomicAdd(&cnt[id + 1], 1);
+  // one atomic per cell and warp: atoms in spatial order share cells within a warp
+  const unsigned peers = __match_any_sync(__activemask(), id);
+  if ((int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&cnt[id + 1], __popc(peers));
 }
 
 // counting-sort placement: cpos[slot] = (x, y, z, i as int bits); order inside a cell is free
@@ -264,7 +266,13 @@ __global__ void k_cell_place(int N, const float* __restrict__ pos, const int* __
   if (i >= N) return;
   const int id = cell_id[i];
   if (id < 0) return;
-  const int slot = cell_start[id] + atomicAdd(&cursor[id], 1);
+  // one atomic per cell and warp; each lane then takes its rank among the warp's atoms of the cell
+  const unsigned peers = __match_any_sync(__activemask(), id);
+  const int lane = threadIdx.x & 31, leader = __ffs(peers) - 1;
+  int base = 0;
+  if (lane == leader) base = atomicAdd(&cursor[id], __popc(peers));
+  base = __shfl_sync(peers, base, leader);
+  const int slot = cell_start[id] + base + __popc(peers & ((1u << lane) - 1u));
   cpos[slot] = make_float4(pos[3 * i], pos[3 * i + 1], pos[3 * i + 2], __int_as_float(i));
 }
 
@@ -492,6 +500,24 @@ __global__ void __launch_bounds__(kPadWarps * 32) k_cell_padded(
   }
 }
 
+// The atoms of each cell in ascending index order, cells in their grid order: perm[k] is the
+// atom at position k (one warp per cell; an atom's place is its rank among the cell's atoms).
+__global__ void k_cell_order(long long cmax, const int* __restrict__ cell_start,
+                             const float4* __restrict__ cpos, int* __restrict__ perm) {
+  const int lane = threadIdx.x & 31;
+  const long long warps = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long c = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; c < cmax;
+       c += warps) {
+    const int a = cell_start[c], b = cell_start[c + 1];
+    for (int k = a + lane; k < b; k += 32) {
+      const int me = __float_as_int(cpos[k].w);
+      int r = 0;
+      for (int o = a; o < b; ++o) r += __float_as_int(cpos[o].w) < me ? 1 : 0;
+      perm[a + r] = me;
+    }
+  }
+}
+
 int sm_count() {
   int dev = 0, n = 148;
   cudaGetDevice(&dev);
@@ -629,4 +655,28 @@ extern "C" int mp_neighbor_padded(int N, const float* pos, const int* graph_ptr,
   if (rc != MP_OK) return rc;
   if (!ok) return MP_ERR_CUDA;
   return host[1] ? MP_ERR_INVALID_ARG : host[0] ? MP_ERR_CAPACITY : MP_OK;
+}
+
+extern "C" int mp_spatial_order(int N, const float* pos, const int* graph_ptr, int n_graphs,
+                                float cell, int* perm, void* stream) {
+  if (N < 0 || (N > 0 && (!pos || !perm)) || !(cell > 0.f) || !std::isfinite(cell) ||
+      (graph_ptr && n_graphs < 1))
+    return MP_ERR_INVALID_ARG;
+  if (N == 0) return MP_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int G = graph_ptr ? n_graphs : 1;
+  Cells c;
+  int rc = build_cells(c, N, pos, graph_ptr, G, cell, s);
+  if (rc == MP_OK) {
+    cudaMemsetAsync(perm, 0xff, sizeof(int) * (size_t)N, s);  // atoms outside every graph: -1
+    k_cell_order<<<sm_count() * 8, 256, 0, s>>>(c.cmax, c.cell_start, c.cpos, perm);
+    if (cudaGetLastError() != cudaSuccess) rc = MP_ERR_CUDA;
+  }
+  int host[2] = {0, 0};
+  if (rc == MP_OK) cudaMemcpyAsync(host, c.flag, 2 * sizeof(int), cudaMemcpyDeviceToHost, s);
+  const bool ok = cudaStreamSynchronize(s) == cudaSuccess && cudaGetLastError() == cudaSuccess;
+  if (c.buf) cudaFreeAsync(c.buf, s);
+  if (rc != MP_OK) return rc;
+  if (!ok) return MP_ERR_CUDA;
+  return host[1] ? MP_ERR_INVALID_ARG : MP_OK;
 }

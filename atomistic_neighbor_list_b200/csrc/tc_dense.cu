@@ -52,6 +52,35 @@ __device__ __forceinline__ void load_a_row(uint8_t* sA, const void* in, bool in_
   }
 }
 
+// Columns [half Kin/2, (half + 1) Kin/2) of row r, the same way: two threads per row share a tile.
+__device__ __forceinline__ void load_a_half(uint8_t* sA, const void* in, bool in_bf16, int Kin, int r,
+                                            bool valid, int lane, int half) {
+  const int k0 = half * (Kin / 2), kn = Kin / 2;  // 32 or 64 columns
+  if (in_bf16) {
+    const uint4* src = (const uint4*)((const __nv_bfloat16*)in + (size_t)r * Kin + k0);
+    uint4 v[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      v[c] = (valid && c < kn / 8) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      if (c < kn / 8) *(uint4*)(sA + kmaj(lane, k0 + 8 * c, Kin)) = v[c];
+  } else {
+    const float4* src = (const float4*)((const float*)in + (size_t)r * Kin + k0);
+    float4 v[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c)
+      v[c] = (valid && c < kn / 4) ? __ldg(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      if (c < kn / 8)
+        *(uint4*)(sA + kmaj(lane, k0 + 8 * c, Kin)) =
+            make_uint4(tc::pack_bf16(v[2 * c].x, v[2 * c].y), tc::pack_bf16(v[2 * c].z, v[2 * c].w),
+                       tc::pack_bf16(v[2 * c + 1].x, v[2 * c + 1].y),
+                       tc::pack_bf16(v[2 * c + 1].z, v[2 * c + 1].w));
+  }
+}
+
 // The readout epilogue for one row: a = acc + d1 over `ncol` columns starting at col; u = dE/da =
 // sigmoid(a) B2 stored, and sum ssp(a) B2 returned.
 __device__ __forceinline__ float readout_cols(const float* v, int col, const float* B2, float* u) {
@@ -189,7 +218,8 @@ __global__ void __launch_bounds__(DTHREADS) k_dense_tc(DenseArgs a, int* status)
   if (warp == 0) tc::tmem_dealloc(tmem, 64);
 }
 
-// Two atomwise layers in one pass over a 128-row tile (thread = row = TMEM lane):
+// Two atomwise layers in one pass over a 128-row tile (two threads per row = TMEM lane, one per
+// half of the columns):
 //   y   = in1 . W1 + b1            (128 columns, fp32): out1 = y (STORE) or out1 += y (RESIDUAL)
 //   out2 = out1_row . W2 + b2      (the updated fp32 row, as bf16, is the second MMA's operand):
 //          STORE -> bf16 [N][128], or READOUT (W2 = B1, 64 columns) -> u [N][64] and e_atom
@@ -213,7 +243,9 @@ struct Dense2Args {
   float* e_atom;
 };
 
-__global__ void __launch_bounds__(DTHREADS) k_dense2_tc(Dense2Args a, int* status) {
+constexpr int D2THREADS = 256;
+
+__global__ void __launch_bounds__(D2THREADS) k_dense2_tc(Dense2Args a, int* status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sW1 = sm;                     // 128 x K1
@@ -222,7 +254,9 @@ __global__ void __launch_bounds__(DTHREADS) k_dense2_tc(Dense2Args a, int* statu
   uint8_t* sA2 = sm + 3 * 128 * 128 * 2; // 128 x 128
   __shared__ uint64_t mbar_w, mbar1, mbar2;
   __shared__ uint32_t tslot;
+  __shared__ float s_e[2][DT];  // readout: the two halves' partial energies of each row
   const int tid = threadIdx.x, warp = tid >> 5;
+  const int lrow = tid & (DT - 1), half = tid >> 7;  // row of the tile, half of the columns
   const int K1 = a.K1, N2 = a.N2;
   if (warp == 0) tc::tmem_alloc(&tslot, 256);
   if (tid == 0) {
@@ -233,15 +267,15 @@ __global__ void __launch_bounds__(DTHREADS) k_dense2_tc(Dense2Args a, int* statu
     tc::bulk_g2s(sW1, a.w1, 128 * K1 * 2, &mbar_w);
     tc::bulk_g2s(sW2, a.w2, N2 * 128 * 2, &mbar_w);
   }
-  const int r = blockIdx.x * DT + tid;
+  const int r = blockIdx.x * DT + lrow;
   const bool valid = r < a.N;
-  load_a_row(sA1, a.in1, a.in1_bf16 != 0, K1, r, valid, tid);
+  load_a_half(sA1, a.in1, a.in1_bf16 != 0, K1, r, valid, lrow, half);
   tc::fence_proxy_async();
   tc::fence_before();
   __syncthreads();
   tc::fence_after();
   const uint32_t tmem = tslot;
-  const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
+  const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
   int bad = 0;
   bool issued1 = false, issued2 = false;  // thread 0: MMAs it has issued
   if (tid == 0) {
@@ -265,7 +299,7 @@ __global__ void __launch_bounds__(DTHREADS) k_dense2_tc(Dense2Args a, int* statu
   if (ok) {
     // ---- first layer's epilogue: the updated row, kept in fp32 and staged as bf16
 #pragma unroll 1
-    for (int c0 = 0; c0 < 128; c0 += 32) {
+    for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
       uint32_t rr[32];
       tc::ld32(lane_base + c0, rr);
       tc::ld_wait();
@@ -291,7 +325,7 @@ __global__ void __launch_bounds__(DTHREADS) k_dense2_tc(Dense2Args a, int* statu
       }
 #pragma unroll
       for (int i = 0; i < 32; i += 8)
-        *(uint4*)(sA2 + kmaj(tid, c0 + i, 128)) =
+        *(uint4*)(sA2 + kmaj(lrow, c0 + i, 128)) =
             valid ? make_uint4(tc::pack_bf16(v[i], v[i + 1]), tc::pack_bf16(v[i + 2], v[i + 3]),
                                tc::pack_bf16(v[i + 4], v[i + 5]), tc::pack_bf16(v[i + 6], v[i + 7]))
                   : make_uint4(0, 0, 0, 0);
@@ -316,7 +350,7 @@ __global__ void __launch_bounds__(DTHREADS) k_dense2_tc(Dense2Args a, int* statu
     // ---- second layer's epilogue
     float e_acc = 0.f;
 #pragma unroll 1
-    for (int c0 = 0; c0 < N2; c0 += 32) {
+    for (int c0 = half * (N2 / 2); c0 < (half + 1) * (N2 / 2); c0 += 32) {
       uint32_t rr[32];
       tc::ld32(lane_base + 128 + c0, rr);
       tc::ld_wait();
@@ -335,7 +369,11 @@ __global__ void __launch_bounds__(DTHREADS) k_dense2_tc(Dense2Args a, int* statu
         }
       }
     }
-    if (a.mode2 == MODE_READOUT && valid) a.e_atom[r] = e_acc + a.d2[0];
+    if (a.mode2 == MODE_READOUT) {  // the two halves' sums, added in a fixed order
+      s_e[half][lrow] = e_acc;
+      __syncthreads();
+      if (half == 0 && valid) a.e_atom[r] = (s_e[0][lrow] + s_e[1][lrow]) + a.d2[0];
+    }
   } else if (tid == 0) {
     raise_status(status, kStatusTimeout);
     // nothing this thread issued may still run when TMEM is freed: the second barrier's first
@@ -419,8 +457,8 @@ int tc_dense2(mp_ctx* ctx, int N, int K1, const void* in1, bool in1_bf16, const 
   const size_t smem = 4 * 128 * 128 * 2 + 1024;
   cudaFuncSetAttribute(k_dense2_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   const int ntiles = (N + DT - 1) / DT;
-  return launch(ctx, K_DENSE_TC, k_dense2_tc, dim3(ntiles > 0 ? ntiles : 1), dim3(DTHREADS), smem, s,
-                a, ctx->status_d);
+  return launch(ctx, K_DENSE_TC, k_dense2_tc, dim3(ntiles > 0 ? ntiles : 1), dim3(D2THREADS), smem,
+                s, a, ctx->status_d);
 }
 
 }  // namespace mp

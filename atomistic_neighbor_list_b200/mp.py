@@ -70,6 +70,7 @@ def _load():
                                vp, vp, vp]),
         "mp_attn_bwd": (i32, [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp]),
         "mp_attn_eq_fwd": (i32, [vp, i32, i32, vp, vp, vp, vp, vp, vp]),
+        "mp_spatial_order": (i32, [i32, vp, vp, i32, c_float, vp, vp]),
         "mp_md_run": (i32, [vp, i32, vp, vp, vp, vp, c_float, i32, vp, vp, i32, c_float, i32,
                             c_float, i32, vp, vp, i64, POINTER(i64), vp, vp, POINTER(i32), vp]),
         "mp_selftest_tc": (i32, [POINTER(i32)]),
@@ -89,7 +90,7 @@ EXPORTED = ("mp_init", "mp_destroy", "mp_strerror", "mp_status_sync", "mp_neighb
             "mp_neighbor_padded", "mp_cfconv_fwd", "mp_attn_fwd", "mp_energy_forces",
             "mp_profile_begin", "mp_profile_end", "mp_profile_get", "mp_launch_count",
             "mp_attn_fwd_noalloc", "mp_selftest_tc", "mp_set_graphs",
-            "mp_md_verlet", "mp_md_run", "mp_attn_bwd", "mp_attn_eq_fwd")
+            "mp_md_verlet", "mp_md_run", "mp_attn_bwd", "mp_attn_eq_fwd", "mp_spatial_order")
 NOALLOC_MAX_NF = 524288  # MP_NOALLOC_MAX_NF: largest N * F mp_attn_fwd_noalloc accepts
 
 
@@ -429,6 +430,20 @@ def neighbor_csr(pos, r_c: float, graph_ptr=None, capacity: int | None = None, s
     _check(lib.mp_neighbor_csr(N, _ptr(pos), _ptr(graph_ptr), G, r_c, _ptr(row_ptr), _ptr(col_idx),
                                capacity, ctypes.byref(n), _stream(stream)), "mp_neighbor_csr")
     return row_ptr, col_idx[: n.value]
+
+
+def spatial_order(pos, cell: float, graph_ptr=None, stream=None):
+    """mp_spatial_order: int32 [N] permutation grouping the atoms of each graph by grid cell."""
+    N = pos.shape[0]
+    _need(pos, "pos", torch.float32, (N, 3))
+    G = 1
+    if graph_ptr is not None:
+        _need(graph_ptr, "graph_ptr", torch.int32)
+        G = graph_ptr.numel() - 1
+    perm = torch.empty(N, dtype=torch.int32, device=pos.device)
+    _check(lib.mp_spatial_order(N, _ptr(pos), _ptr(graph_ptr), G, float(cell), _ptr(perm),
+                                _stream(stream)), "mp_spatial_order")
+    return perm
 
 
 def neighbor_padded(pos, r_c: float, K: int, graph_ptr=None, stream=None):

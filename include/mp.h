@@ -143,6 +143,18 @@ int mp_neighbor_csr(int N, const float* pos, const int* graph_ptr, int n_graphs,
 int mp_neighbor_padded(int N, const float* pos, const int* graph_ptr, int n_graphs, float r_c,
                        int K, int* nbr, unsigned char* mask, void* stream);
 
+/* A spatial order of the atoms for locality of the row gathers [TS: atoms organised along a
+ * space-filling curve]: perm[k] = index of the atom placed at position k. Within each graph the
+ * atoms are grouped by cell of the grid mp_neighbor_csr uses (cells at least `cell` wide over the
+ * graph's bounding box, visited x fastest, then y, then z), atoms of a cell in ascending index
+ * order; graphs keep their ranges, so graph_ptr stays valid for the permuted system. A caller
+ * that applies the permutation to its per-atom arrays (positions, types, velocities, features)
+ * gets the same physics with neighbors close in memory (the energy and forces are those of the
+ * relabelled system). perm: int32 [N] (device). Synchronises `stream`.
+ * Errors: MP_ERR_INVALID_ARG, MP_ERR_CAPACITY, MP_ERR_CUDA.                                    */
+int mp_spatial_order(int N, const float* pos, const int* graph_ptr, int n_graphs, float cell,
+                     int* perm, void* stream);
+
 /* One continuous-filter convolution [FS s.2.1-2.3] with block `block`'s filter weights:
  *   out_i = sum_{j in row i} x_j (.) W(|r_i - r_j|),   rows with no edges give 0.
  * x, out: [N][F] of the context dtype (float or bf16), 16-byte aligned (rows are read and

@@ -130,3 +130,46 @@ def test_padded_row_beyond_staging_is_a_capacity_error(mp):
     with pytest.raises(mp.MpError) as e:
         mp.neighbor_padded(dev(pos), 5.0, 8)
     assert e.value.name == "MP_ERR_CAPACITY"
+
+
+def test_spatial_order_is_a_graph_preserving_permutation(mp):
+    """mp_spatial_order: a permutation that keeps every atom inside its graph's range and places
+    neighbors close together; the energy and forces of the relabelled system are the original
+    ones, relabelled."""
+    wl = synth.WORKLOADS["cfg3"]
+    import dataclasses
+    wl = dataclasses.replace(wl, n_atoms=4 * 300, replicas=4)
+    pos, gp = synth.positions_for(wl)
+    perm = mp.spatial_order(dev(pos), wl.r_c, graph_ptr=dev(gp)).cpu().numpy()
+    assert np.array_equal(np.sort(perm), np.arange(len(pos)))
+    for g in range(len(gp) - 1):
+        seg = perm[gp[g]:gp[g + 1]]
+        assert seg.min() >= gp[g] and seg.max() < gp[g + 1]
+    # locality: consecutive atoms of the new order are much closer than in the old one
+    p2 = pos[perm]
+    step_new = np.linalg.norm(np.diff(p2, axis=0), axis=1).mean()
+    u = synth.uniform_positions(5000, seed=3)
+    pu = u[mp.spatial_order(dev(u), 5.0).cpu().numpy()]
+    assert np.linalg.norm(np.diff(pu, axis=0), axis=1).mean() < 0.25 * np.linalg.norm(
+        np.diff(u, axis=0), axis=1).mean()
+    assert np.isfinite(step_new)
+
+
+def test_spatial_order_relabels_energy_and_forces(mp):
+    import dataclasses
+    wl = dataclasses.replace(synth.scaled(synth.WORKLOADS["cfg2"], 2000), dtype="fp32")
+    pos, _ = synth.positions_for(wl)
+    types = synth.atom_types(len(pos), wl.n_types)
+    perm = mp.spatial_order(dev(pos), wl.r_c).cpu().numpy()
+    out = []
+    for p, t in ((pos, types), (pos[perm], types[perm])):
+        pd = dev(np.ascontiguousarray(p))
+        rp, ci = mp.neighbor_csr(pd, wl.r_c)
+        ctx = mp.Context.from_workload(wl, synth.make_weights(wl), max_atoms=len(p),
+                                       max_edges=ci.numel())
+        e, f = ctx.energy_forces(pd, dev(np.ascontiguousarray(t)), rp, ci)
+        torch.cuda.synchronize()
+        out.append((float(e[0]), f.cpu().numpy()))
+    (e0, f0), (e1, f1) = out
+    assert abs(e0 - e1) <= 1e-5 * abs(e0)
+    assert np.abs(f1 - f0[perm]).max() <= 1e-4 * np.abs(f0).max()
