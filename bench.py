@@ -490,13 +490,18 @@ def main():
                   col_idx=ci_r, rebuild_every=10, max_disp=0.25, check_every=1)
         ctx_md.md_run(p_md, vel, types_d, 10, dt, skin, cap, **kw)
         torch.cuda.synchronize()
-        t0 = time.perf_counter()
-        res_r = ctx_md.md_run(p_md, vel, types_d, md_steps, dt, skin, cap, **kw)
-        torch.cuda.synchronize()
-        ms_r = (time.perf_counter() - t0) * 1000.0 / md_steps
+        runs = []
+        for _ in range(3):  # the median of three calls: each synchronises the host every step
+            t0 = time.perf_counter()
+            res_r = ctx_md.md_run(p_md, vel, types_d, md_steps, dt, skin, cap, **kw)
+            torch.cuda.synchronize()
+            runs.append((time.perf_counter() - t0) * 1000.0 / md_steps)
+        ms_r = sorted(runs)[1]
         md["with_rebuilds"] = {
             "value": 1000.0 / ms_r, "unit": "MD steps/s", "ms_per_step": ms_r,
-            "builds": res_r["n_builds"], "timing": "host wall clock (the call synchronises)",
+            "builds": res_r["n_builds"],
+            "timing": "host wall clock (the call synchronises), median of 3 calls",
+            "ms_per_step_runs": runs,
             "policy": "list at r_c + 0.5 A rebuilt every 10 steps or when an atom moved 0.25 A "
                       "(checked every step); energy and forces re-evaluated after each build"}
         # one neighbor-list construction at the workload's cutoff (host wall clock: it synchronises)
