@@ -5,23 +5,24 @@
 //   [z1 | bias] = e [A1ext | P],  [t | b'] = e' [A1 | P]                  (MMA1, N = 144 each)
 //   v = (sigmoid(z1) t) A2,  u = ssp(z1) A2                              (MMA2b, MMA2a)
 //   W = f_c (u + c2),  W' = f_c' (u + c2) + f_c v
-// and, per slot s of row i and head h, in the epilogue (thread = slot, half of the features):
+// and, per slot s of row i and head h, in the epilogue (thread = slot, a quarter of the features):
 //   l = q_i . k_j / sqrt(8) + bias,  dalpha = sum g_i x_j W,  beta = sum g_i x_j W',  b'.
 // Once the row's K / 128 tiles are done: the row's softmax statistics (max, sum, D = sum alpha
 // dalpha), dL/dq_i = sum_s dl k_j / sqrt(8) and the row side of dL/dr_i, as the CUDA-core pass.
-// One CTA of 256 threads per SM, lock-step tiles; every wait is bounded.
+// One CTA of 512 threads per SM (four warps per TMEM lane quarter), lock-step tiles; every wait
+// is bounded.
 #include "tc_common.cuh"
 
 namespace mp {
 namespace {
 using namespace tcc;
 
-constexpr int BT = 256;          // threads
+constexpr int BT = 512;          // threads: four warps per TMEM lane quarter
 constexpr int BH = 16, BD = 8;   // heads, head width
 constexpr int BN1 = FT + BH;     // MMA1 columns: the filter's first layer and the radial bias
 constexpr int KMAX = 256;        // slots per row this kernel keeps on chip
-constexpr int SLS = KMAX + 16;   // row stride of the per-head slot arrays (the two half warps of
-                                 // a statistics pass land on disjoint banks)
+constexpr int SLS = KMAX + 16;   // row stride of the per-head slot arrays (rows of consecutive
+                                 // heads start on different banks)
 
 struct BwSmem {
   uint32_t w1, w2, c2, x, row, total;
@@ -47,14 +48,14 @@ __host__ __device__ constexpr bool bw_fits_attn(int K1) {
 }
 
 // The filter of a tile's 128 entries and its d-derivative on the tensor cores. Every thread of
-// the CTA calls it with its entry e (TMEM lane), feature half, distance d and validity; on return
+// the CTA calls it with its entry e (TMEM lane), feature quarter, distance d and validity; on return
 // (all MMAs complete) TMEM holds u = ssp(z1) A2 in columns [0,128), the radial bias of the 16
 // heads in [128,144), v = (sigmoid(z1) t) A2 in [256,384) and the bias's d-derivative in
 // [384,400). The operand area sX is free again. False when a bounded wait ran out.
 template <int K1>
 __device__ __forceinline__ bool filter_tile(uint8_t* sX, uint32_t sX_a, uint32_t sW1_a,
                                             uint32_t sW2_a, uint32_t tmem, uint32_t lane_base,
-                                            int e, int half, float d, bool ok, const Radial& rp,
+                                            int e, int part, float d, bool ok, const Radial& rp,
                                             uint64_t* mbar, uint32_t& phase) {
   const int tid = threadIdx.x;
   auto wait_mma = [&]() -> bool {
@@ -66,12 +67,16 @@ __device__ __forceinline__ bool filter_tile(uint8_t* sX, uint32_t sX_a, uint32_t
   const uint32_t id1 = tc::idesc(TM, BN1, 1, false, false);
   const uint32_t id2 = tc::idesc(TM, FT, 1, false, false);
   const float nglog2e = -rp.gamma * LOG2E;
-  // half 0 writes the Gaussian row e (with the constant bias column), half 1 e' = de/dd
+  // parts 0 and 1 write the two halves of the Gaussian row e (with the constant bias column),
+  // parts 2 and 3 those of e' = de/dd
   {
     const float d0 = d - rp.mu_min;
-    uint8_t* dstA = sX + half * (TM * K1 * 2);
+    const bool deriv = part >= 2;
+    uint8_t* dstA = sX + (deriv ? TM * K1 * 2 : 0);
+    const int kb = (part & 1) * (K1 / 2);
 #pragma unroll
-    for (int k0 = 0; k0 < K1; k0 += 8) {
+    for (int c8 = 0; c8 < K1 / 16; ++c8) {
+      const int k0 = kb + 8 * c8;
       uint32_t w[4];
 #pragma unroll
       for (int qq = 0; qq < 4; ++qq) {
@@ -82,7 +87,7 @@ __device__ __forceinline__ bool filter_tile(uint8_t* sX, uint32_t sX_a, uint32_t
           const float dd = fmaf(-(float)k, rp.dmu, d0);
           const float ek = tc::ex2f(nglog2e * dd * dd);
           float val;
-          if (half == 0) val = k < rp.R ? ek : (k == rp.R ? 1.f : 0.f);
+          if (!deriv) val = k < rp.R ? ek : (k == rp.R ? 1.f : 0.f);
           else val = k < rp.R ? -2.f * rp.gamma * dd * ek : 0.f;
           v[hh] = ok ? val : 0.f;
         }
@@ -108,9 +113,8 @@ __device__ __forceinline__ bool filter_tile(uint8_t* sX, uint32_t sX_a, uint32_t
   }
   if (!wait_mma()) return false;
   // E1a: Q = sigmoid(z1) t
-#pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    const int f0 = 64 * half + 32 * c;
+  {
+    const int f0 = 32 * part;
     uint32_t rz[32], rt[32];
     tc::ld32(lane_base + f0, rz);
     tc::ld32(lane_base + 256 + f0, rt);
@@ -144,9 +148,8 @@ __device__ __forceinline__ bool filter_tile(uint8_t* sX, uint32_t sX_a, uint32_t
   }
   if (!wait_mma()) return false;
   // E1b: P = ssp(z1)
-#pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    const int f0 = 64 * half + 32 * c;
+  {
+    const int f0 = 32 * part;
     uint32_t rz[32];
     tc::ld32(lane_base + f0, rz);
     tc::ld_wait();
@@ -227,7 +230,7 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_dst_tc(
   bool aborted = __syncthreads_or(tc::mbar_wait(&s_mbar[1], 0, WAIT_LIMIT) ? 0 : 1) != 0;
   const uint32_t sX_a = tc::smem_u32(sX), sW1_a = tc::smem_u32(sW1), sW2_a = tc::smem_u32(sW2);
   // TMEM columns: [0,144) z1 | bias, then u in [0,128); [256,400) t | b', then v in [256,384)
-  const int q4 = warp & 3, half = warp >> 2;  // lane quarter; features [64 half, 64 half + 64)
+  const int q4 = warp & 3, part = warp >> 2;  // lane quarter; features [32 part, 32 part + 32)
   const int e = 32 * q4 + lane;               // the tile's slot this thread works on
   const uint32_t lane_base = tmem + ((uint32_t)(32 * q4) << 16);
 
@@ -245,7 +248,7 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_dst_tc(
         int j = nbr[slot];
         bool ok = mask[slot] != 0;
         if (ok && (unsigned)j >= (unsigned)N) {
-          if (half == 0) raise_status(status, kStatusBounds);
+          if (part == 0) raise_status(status, kStatusBounds);
           ok = false;
         }
         if (!ok) j = 0;
@@ -262,7 +265,7 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_dst_tc(
             uz = dz * inv;
           }
         }
-        if (half == 0) {
+        if (part == 0) {
           s_src[s0 + e] = ok ? j : -1;
           s_u[3 * (s0 + e)] = ux;
           s_u[3 * (s0 + e) + 1] = uy;
@@ -271,7 +274,7 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_dst_tc(
           s_dfc[e] = dfc;
           s_tj[e] = j;
         }
-        if (!filter_tile<K1>(sX, sX_a, sW1_a, sW2_a, tmem, lane_base, e, half, d, ok, rp,
+        if (!filter_tile<K1>(sX, sX_a, sW1_a, sW2_a, tmem, lane_base, e, part, d, ok, rp,
                              &s_mbar[0], phase)) {
           aborted = true;
           break;
@@ -283,14 +286,16 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_dst_tc(
         const float fc = s_fc[e], dfc = s_dfc[e];
         const bool ok = s_src[s0 + e] >= 0;
         uint32_t rb[8], rp8[8];
-        tc::ld8(lane_base + FT + 8 * half, rb);        // the radial bias of heads 8 half ..
-        tc::ld8(lane_base + 256 + FT + 8 * half, rp8);  // and its d-derivative b'
+        tc::ld8(lane_base + FT + 8 * (part >> 1), rb);        // the radial bias of 8 heads ..
+        tc::ld8(lane_base + 256 + FT + 8 * (part >> 1), rp8);  // and its d-derivative b'
         tc::ld_wait(rb, rp8);
         const __nv_bfloat16* xr = x + (size_t)j * FT;
         const float* kr = kx + (size_t)j * FT;
 #pragma unroll
-        for (int hh = 0; hh < 8; ++hh) {  // head 8 half + hh: features f0 .. f0 + 7
-          const int f0 = 64 * half + 8 * hh;
+        for (int hh = 0; hh < 4; ++hh) {  // head 4 part + hh: features f0 .. f0 + 7
+          const int f0 = 32 * part + 8 * hh;
+          const float bias_h = __uint_as_float((part & 1) ? rb[4 + hh] : rb[hh]);
+          const float bp_h = __uint_as_float((part & 1) ? rp8[4 + hh] : rp8[hh]);
           uint32_t ru[8], rv[8];
           tc::ld8(lane_base + f0, ru);
           tc::ld8(lane_base + 256 + f0, rv);
@@ -313,11 +318,11 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_dst_tc(
             be = fmaf(gx, Wp, be);
           }
           if (ok) {
-            const int o = (8 * half + hh) * SLS + s0 + e;
-            s_l[o] = l + __uint_as_float(rb[hh]);
+            const int o = (4 * part + hh) * SLS + s0 + e;
+            s_l[o] = l + bias_h;
             s_da[o] = da;
             s_be[o] = be;
-            s_bp[o] = __uint_as_float(rp8[hh]);
+            s_bp[o] = bp_h;
           }
         }
       }
@@ -326,22 +331,22 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_dst_tc(
     }
     if (aborted) break;
     // ------------------------------------------------------------------ the row's statistics
-    // 16 threads per head (a half warp), slots strided over them
+    // one warp per head, slots strided over its lanes
     {
-      const int h = tid >> 4, c = tid & 15;
+      const int h = warp, c = lane;
       float m = -INFINITY;
-      for (int s = c; s < K; s += 16)
+      for (int s = c; s < K; s += 32)
         if (s_src[s] >= 0) m = fmaxf(m, s_l[h * SLS + s]);
-      for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
       float z = 0.f;
-      for (int s = c; s < K; s += 16)
+      for (int s = c; s < K; s += 32)
         if (s_src[s] >= 0) z += tc::ex2f((s_l[h * SLS + s] - m) * LOG2E);
-      for (int o = 8; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+      for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
       const float iz = z > 0.f ? 1.f / z : 0.f;
       float D = 0.f;
-      for (int s = c; s < K; s += 16)
+      for (int s = c; s < K; s += 32)
         if (s_src[s] >= 0) D += tc::ex2f((s_l[h * SLS + s] - m) * LOG2E) * iz * s_da[h * SLS + s];
-      for (int o = 8; o > 0; o >>= 1) D += __shfl_xor_sync(0xffffffffu, D, o);
+      for (int o = 16; o > 0; o >>= 1) D += __shfl_xor_sync(0xffffffffu, D, o);
       if (c == 0) {
         s_st[h] = m;
         s_st[BH + h] = iz;
@@ -352,22 +357,23 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_dst_tc(
       }
     }
     __syncthreads();
-    // dL/dq_i: thread (feature f, parity) sums every other slot; the two halves meet in smem
+    // dL/dq_i: thread (feature f, residue r of the slot mod 4) sums a quarter of the slots; the
+    // four partial sums meet in shared memory and are added in a fixed order
     {
       const int f = tid & (FT - 1), par = tid >> 7, h = f >> 3;
       const float m = s_st[h], iz = s_st[BH + h], D = s_st[2 * BH + h];
       float acc = 0.f;
-      for (int s0 = par; s0 < K; s0 += 16) {  // eight independent gathers in flight
+      for (int s0 = par; s0 < K; s0 += 32) {  // eight independent gathers in flight
         float kv[8];
 #pragma unroll
         for (int u8 = 0; u8 < 8; ++u8) {
-          const int s = s0 + 2 * u8;
+          const int s = s0 + 4 * u8;
           const int j = s < K ? s_src[s] : -1;
           kv[u8] = j >= 0 ? kx[(size_t)j * FT + f] : 0.f;
         }
 #pragma unroll
         for (int u8 = 0; u8 < 8; ++u8) {
-          const int s = s0 + 2 * u8;
+          const int s = s0 + 4 * u8;
           if (s < K && s_src[s] >= 0) {
             const int o = h * SLS + s;
             const float a = tc::ex2f((s_l[o] - m) * LOG2E) * iz;
@@ -375,10 +381,11 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_dst_tc(
           }
         }
       }
-      float* part = (float*)sX;      // the operand area is free between rows
-      if (par == 1) part[f] = acc;
+      float* pacc = (float*)sX;      // the operand area is free between rows
+      if (par > 0) pacc[par * FT + f] = acc;
       __syncthreads();
-      if (par == 0) gq[(size_t)i * FT + f] = (acc + part[f]) * qscale;
+      if (par == 0)
+        gq[(size_t)i * FT + f] = (((acc + pacc[FT + f]) + pacc[2 * FT + f]) + pacc[3 * FT + f]) * qscale;
     }
     // dL/dr_i, row side: each slot's dL/dd over the heads times (r_i - r_j) / d
     {
@@ -402,14 +409,14 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_dst_tc(
         gp2 += __shfl_xor_sync(0xffffffffu, gp2, o);
       }
       if (lane == 0) {
-        s_red[8 + warp] = gp0;
-        s_red[16 + warp] = gp1;
-        s_red[24 + warp] = gp2;
+        s_red[16 + warp] = gp0;
+        s_red[32 + warp] = gp1;
+        s_red[48 + warp] = gp2;
       }
       __syncthreads();
       if (tid < 3) {
         float v = 0.f;
-        for (int w = 0; w < BT / 32; ++w) v += s_red[8 * (tid + 1) + w];
+        for (int w = 0; w < BT / 32; ++w) v += s_red[16 * (tid + 1) + w];
         grad_pos[3 * i + tid] = v;
       }
       __syncthreads();  // s_q, s_g, the slot data and the operand area are reused by the next row
@@ -422,9 +429,9 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_dst_tc(
 }
 
 // ------------------------------------------------------------------------------ source pass
-// One CTA of 256 threads per SM; per source atom j, its transposed entries (row i, slot), in
+// One CTA of 512 threads per SM; per source atom j, its transposed entries (row i, slot), in
 // ascending order, in tiles of 128: the filter as in the destination pass; then per entry and head
-// (thread = entry, half of the features) alpha = e^(l - m_ih) / z_ih from the row's statistics,
+// (thread = entry, a quarter of the features) alpha = e^(l - m_ih) / z_ih from the row's statistics,
 // dalpha, beta and dl = alpha (dalpha - D_ih); per feature the entry's terms dl q_i / sqrt(8) (of
 // dL/dk_j) and alpha g_i W (the value path of dL/dx_j), summed over the entries by two MMAs of
 // bf16 message tiles against a column of ones, accumulated in TMEM over the source's tiles; and
@@ -443,9 +450,9 @@ __host__ __device__ constexpr SrSmem sr_layout(int K1) {
   L.m2 = o;   o += FT * TM * 2;
   L.ones = o; o += 16 * TM * 2;
   L.misc = o;
-  // k_j, x_j [F]; per entry: row, envelope, its derivative, unit vector [3], two dL/dd halves;
+  // k_j, x_j [F]; per entry: row, envelope, its derivative, unit vector [3], four dL/dd parts;
   // reduction scratch; mbarriers and the TMEM slot
-  o += 2 * FT * 4 + TM * (1 + 2 + 3 + 2) * 4 + 64 * 4 + 64;
+  o += 2 * FT * 4 + TM * (1 + 2 + 3 + 4) * 4 + 64 * 4 + 64;
   L.total = o;
   return L;
 }
@@ -475,8 +482,8 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_src_tc(
   float* s_fc = (float*)(s_row + TM);  // [TM]
   float* s_dfc = s_fc + TM;            // [TM]
   float* s_u = s_dfc + TM;             // [TM][3]
-  float* s_sd = s_u + 3 * TM;          // [2][TM] dL/dd of the entry, per feature half
-  float* s_red = s_sd + 2 * TM;        // [64]
+  float* s_sd = s_u + 3 * TM;          // [4][TM] dL/dd of the entry, per feature quarter
+  float* s_red = s_sd + 4 * TM;        // [64]
   uint64_t* s_mbar = (uint64_t*)(s_red + 64);
   uint32_t* s_tmem = (uint32_t*)(s_mbar + 2);
 
@@ -503,7 +510,7 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_src_tc(
   const uint32_t sM1_a = tc::smem_u32(sM1), sM2_a = tc::smem_u32(sM2);
   const uint32_t sOnes_a = tc::smem_u32(sOnes);
   const uint32_t id3 = tc::idesc(TM, 16, 1, true, false);
-  const int q4 = warp & 3, half = warp >> 2;
+  const int q4 = warp & 3, part = warp >> 2;
   const int e = 32 * q4 + lane;
   const uint32_t lane_base = tmem + ((uint32_t)(32 * q4) << 16);
   // TMEM columns [400,416): dL/dk_j per feature (lane); [416,432): the value path of dL/dx_j
@@ -532,7 +539,7 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_src_tc(
       if (ok) {
         i = rev[idx] / K;
         if ((unsigned)i >= (unsigned)N) {
-          if (half == 0) raise_status(status, kStatusBounds);
+          if (part == 0) raise_status(status, kStatusBounds);
           ok = false;
           i = 0;
         }
@@ -550,7 +557,7 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_src_tc(
           uz = dz * inv;
         }
       }
-      if (half == 0) {
+      if (part == 0) {
         s_row[e] = ok ? i : -1;
         s_fc[e] = fc;
         s_dfc[e] = dfc;
@@ -560,7 +567,7 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_src_tc(
         // the ones column: entry e of row 0 of the (slot x entry) matrix
         *(__nv_bfloat16*)(sOnes + kmaj(0, e, TM)) = __float2bfloat16_rn(ok ? 1.f : 0.f);
       }
-      if (!filter_tile<K1>(sX, sX_a, sW1_a, sW2_a, tmem, lane_base, e, half, d, ok, rp,
+      if (!filter_tile<K1>(sX, sX_a, sW1_a, sW2_a, tmem, lane_base, e, part, d, ok, rp,
                            &s_mbar[0], phase)) {
         aborted = true;
         break;
@@ -572,16 +579,18 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_src_tc(
         const int ii = eok ? row : 0;
         const float efc = s_fc[e], edfc = s_dfc[e];
         uint32_t rb[8], rp8[8];
-        tc::ld8(lane_base + FT + 8 * half, rb);
-        tc::ld8(lane_base + 256 + FT + 8 * half, rp8);
+        tc::ld8(lane_base + FT + 8 * (part >> 1), rb);
+        tc::ld8(lane_base + 256 + FT + 8 * (part >> 1), rp8);
         tc::ld_wait(rb, rp8);
         const float* qr = q + (size_t)ii * FT;
         const float* gr = g + (size_t)ii * FT;
         const float* st = stats + (size_t)ii * 3 * BH;
         float sd = 0.f;
 #pragma unroll
-        for (int hh = 0; hh < 8; ++hh) {
-          const int h = 8 * half + hh, f0 = 8 * h;
+        for (int hh = 0; hh < 4; ++hh) {
+          const int h = 4 * part + hh, f0 = 8 * h;
+          const float bias_h = __uint_as_float((part & 1) ? rb[4 + hh] : rb[hh]);
+          const float bp_h = __uint_as_float((part & 1) ? rp8[4 + hh] : rp8[hh]);
           uint32_t ru[8], rv[8];
           tc::ld8(lane_base + f0, ru);
           tc::ld8(lane_base + 256 + f0, rv);
@@ -602,10 +611,10 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_src_tc(
             da = fmaf(gx, W[cc], da);
             be = fmaf(gx, Wp, be);
           }
-          l += __uint_as_float(rb[hh]);
+          l += bias_h;
           const float a = (eok && z > 0.f) ? tc::ex2f((l - m) * LOG2E) * (1.f / z) : 0.f;
           const float dl = a * (da - D);
-          sd = fmaf(a, be, fmaf(dl, __uint_as_float(rp8[hh]), sd));
+          sd = fmaf(a, be, fmaf(dl, bp_h, sd));
           uint32_t w1[4], w2[4];
 #pragma unroll
           for (int c2i = 0; c2i < 4; ++c2i) {
@@ -617,7 +626,7 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_src_tc(
           *(uint4*)(sM1 + mo) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
           *(uint4*)(sM2 + mo) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
         }
-        s_sd[half * TM + e] = eok ? sd : 0.f;
+        s_sd[part * TM + e] = eok ? sd : 0.f;
       }
       tc::fence_proxy_async();
       tc::fence_before();
@@ -642,8 +651,8 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_src_tc(
           break;
         }
       }
-      if (half == 0 && s_row[e] >= 0) {  // -dL/dd (r_i - r_j) / d of this entry
-        const float sdd = s_sd[e] + s_sd[TM + e];
+      if (part == 0 && s_row[e] >= 0) {  // -dL/dd (r_i - r_j) / d of this entry
+        const float sdd = ((s_sd[e] + s_sd[TM + e]) + s_sd[2 * TM + e]) + s_sd[3 * TM + e];
         gp0 = fmaf(-sdd, s_u[3 * e], gp0);
         gp1 = fmaf(-sdd, s_u[3 * e + 1], gp1);
         gp2 = fmaf(-sdd, s_u[3 * e + 2], gp2);
@@ -665,15 +674,15 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_src_tc(
       gp2 += __shfl_xor_sync(0xffffffffu, gp2, o);
     }
     if (lane == 0) {
-      s_red[8 + warp] = gp0;
-      s_red[16 + warp] = gp1;
-      s_red[24 + warp] = gp2;
+      s_red[16 + warp] = gp0;
+      s_red[32 + warp] = gp1;
+      s_red[48 + warp] = gp2;
     }
     tc::fence_before();
     __syncthreads();
     if (tid < 3) {
       float v = 0.f;
-      for (int w = 0; w < BT / 32; ++w) v += s_red[8 * (tid + 1) + w];
+      for (int w = 0; w < BT / 32; ++w) v += s_red[16 * (tid + 1) + w];
       grad_pos[3 * j + tid] += v;  // the destination pass wrote the row side
     }
     __syncthreads();
