@@ -467,7 +467,7 @@ template <typename T, int F>
 int run_attn_bwd(mp_ctx* c, int N, int K, const float* pos, const int* nbr,
                  const unsigned char* mask, const void* x, const float* g, float* grad_x,
                  float* grad_pos, const int* rev_ptr, const int* rev, cudaStream_t s) {
-  const int H = c->cfg.n_heads, D = c->cfg.head_dim, R = c->cfg.n_rbf;
+  const int H = c->cfg.n_heads, D = c->cfg.head_dim;
   const size_t smem_dst = (4 * (size_t)K * H + 3 * (size_t)K) * 4 + (size_t)K * 4;
   auto kd = k_attn_bwd_dst<T, F>;
   auto ks = k_attn_bwd_src<T, F>;
@@ -542,7 +542,7 @@ extern "C" int mp_attn_bwd(mp_ctx* c, int N, int K, const float* pos, const int*
   const int nb = scan_blocks(N) > 0 ? scan_blocks(N) : 1;
   const size_t bytes = 4 * ((size_t)(N + 1) + (size_t)N + 2 * (size_t)NK) + 8 * (size_t)nb + 16;
   char* buf = nullptr;
-  if (cudaMallocAsync((void**)&buf, bytes, s) != cudaSuccess) return MP_ERR_CUDA;
+  if (scratch_alloc((void**)&buf, bytes, s) != cudaSuccess) return MP_ERR_CUDA;
   int* rev_ptr = (int*)buf;
   int* cursor = rev_ptr + N + 1;
   int* tmp = cursor + N;
@@ -575,6 +575,6 @@ extern "C" int mp_attn_bwd(mp_ctx* c, int N, int K, const float* pos, const int*
     else
       rc = MP_ERR_INVALID_ARG;
   }
-  cudaFreeAsync(buf, s);
+  scratch_free(buf, s);
   return rc;
 }

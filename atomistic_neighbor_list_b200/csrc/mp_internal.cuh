@@ -201,6 +201,12 @@ int launch_attn_simt(mp_ctx*, int N, int K, const float* pos, const int* nbr,
                      const unsigned char* mask, const void* x, void* out, cudaStream_t);
 int launch_validate_csr(mp_ctx*, int N, long long E, const int* row_ptr, const int* col_idx,
                         const int* graph_ptr, int n_graphs, bool need_sym, cudaStream_t);
+// Stream-ordered scratch of the context-free calls (neighbor lists, the attention backward's
+// transposed list) from a memory pool of the library's own per device that keeps its memory
+// between calls (the default pool returns memory at each synchronisation, and mapping it again
+// costs more than the kernels it serves). The pool holds at most the largest scratch used.
+cudaError_t scratch_alloc(void** p, size_t bytes, cudaStream_t s);
+void scratch_free(void* p, cudaStream_t s);
 // In place on the stream: a[1..n] counts -> a[0..n] prefix sums (a[0] = 0); *overflow = 1 when the
 // total passes INT_MAX. bsum: scan_blocks(n) (at least 1) long longs of scratch (neighbors.cu).
 int scan_blocks(long long n);

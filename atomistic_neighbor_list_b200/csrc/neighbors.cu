@@ -10,6 +10,7 @@
 // more hits than the staging holds is filled by an ordered scan over its whole graph instead.
 // The result is bit-identical to any implementation of the same rule.
 #include <cmath>
+#include <mutex>
 
 #include "mp_internal.cuh"
 
@@ -137,6 +138,41 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_add(long long n, int* __r
 }  // namespace
 
 int scan_blocks(long long n) { return (int)((n + kScanPer - 1) / kScanPer); }
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_pool_mu;
+cudaMemPool_t g_pool[kMaxDevices] = {};
+}  // namespace
+
+cudaError_t scratch_alloc(void** p, size_t bytes, cudaStream_t s) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= kMaxDevices) return cudaMallocAsync(p, bytes, s);
+  cudaMemPool_t pool;
+  {
+    std::lock_guard<std::mutex> lock(g_pool_mu);
+    if (!g_pool[dev]) {
+      cudaMemPoolProps props{};
+      props.allocType = cudaMemAllocationTypePinned;
+      props.location.type = cudaMemLocationTypeDevice;
+      props.location.id = dev;
+      if ((err = cudaMemPoolCreate(&g_pool[dev], &props)) != cudaSuccess) {
+        g_pool[dev] = nullptr;
+        return err;
+      }
+      uint64_t keep = ~0ull;  // never return memory to the device on synchronisation
+      cudaMemPoolSetAttribute(g_pool[dev], cudaMemPoolAttrReleaseThreshold, &keep);
+    }
+    pool = g_pool[dev];
+  }
+  return cudaMallocFromPoolAsync(p, bytes, pool, s);
+}
+
+void scratch_free(void* p, cudaStream_t s) {
+  if (p) cudaFreeAsync(p, s);
+}
 
 // bsum: scan_blocks(n) (at least 1) long longs of scratch
 void launch_scan(long long n, int* a, long long* bsum, int* overflow, cudaStream_t s) {
@@ -559,7 +595,7 @@ int build_cells(Cells& c, int N, const float* pos, const int* gp, int G, float r
                sz_bsum = align16(8 * (size_t)nb), sz_flag = 16;
   const size_t total =
       sz_grid + sz_off + sz_start + sz_cur + sz_info + sz_id + sz_cpos + sz_bsum + sz_flag;
-  if (cudaMallocAsync(&c.buf, total, s) != cudaSuccess) return MP_ERR_CUDA;
+  if (scratch_alloc(&c.buf, total, s) != cudaSuccess) return MP_ERR_CUDA;
   char* p = (char*)c.buf;
   c.grids = (CellGrid*)p, p += sz_grid;
   c.cell_off = (int*)p, p += sz_off;
@@ -606,7 +642,7 @@ extern "C" int mp_neighbor_csr(int N, const float* pos, const int* graph_ptr, in
   Cells c;
   int rc = build_cells(c, N, pos, graph_ptr, G, r_c, s);
   if (rc != MP_OK) {
-    if (c.buf) cudaFreeAsync(c.buf, s);
+    if (c.buf) scratch_free(c.buf, s);
     return rc;
   }
   const int grid = sm_count() * 8;
@@ -618,7 +654,7 @@ extern "C" int mp_neighbor_csr(int N, const float* pos, const int* graph_ptr, in
   cudaMemcpyAsync(&host[0], row_ptr + N, sizeof(int), cudaMemcpyDeviceToHost, s);
   cudaMemcpyAsync(&host[1], c.flag, 2 * sizeof(int), cudaMemcpyDeviceToHost, s);
   if (cudaStreamSynchronize(s) != cudaSuccess || cudaGetLastError() != cudaSuccess) {
-    cudaFreeAsync(c.buf, s);
+    scratch_free(c.buf, s);
     return MP_ERR_CUDA;
   }
   *n_edges = host[0];
@@ -627,7 +663,7 @@ extern "C" int mp_neighbor_csr(int N, const float* pos, const int* graph_ptr, in
     k_cell_fill<<<sm_count() * 4, kFillWarps * 32, 0, s>>>(N, pos, graph_ptr, G, c.cellinfo,
                                                            c.grids, c.cell_off, c.cell_start,
                                                            c.cpos, rc2, row_ptr, col_idx, capacity);
-  cudaFreeAsync(c.buf, s);
+  scratch_free(c.buf, s);
   if (rc != MP_OK) return rc;
   return cudaGetLastError() == cudaSuccess ? MP_OK : MP_ERR_CUDA;
 }
@@ -651,7 +687,7 @@ extern "C" int mp_neighbor_padded(int N, const float* pos, const int* graph_ptr,
   int host[2] = {0, 0};
   if (rc == MP_OK) cudaMemcpyAsync(host, c.flag, 2 * sizeof(int), cudaMemcpyDeviceToHost, s);
   const bool ok = cudaStreamSynchronize(s) == cudaSuccess && cudaGetLastError() == cudaSuccess;
-  if (c.buf) cudaFreeAsync(c.buf, s);
+  if (c.buf) scratch_free(c.buf, s);
   if (rc != MP_OK) return rc;
   if (!ok) return MP_ERR_CUDA;
   return host[1] ? MP_ERR_INVALID_ARG : host[0] ? MP_ERR_CAPACITY : MP_OK;
@@ -675,7 +711,7 @@ extern "C" int mp_spatial_order(int N, const float* pos, const int* graph_ptr, i
   int host[2] = {0, 0};
   if (rc == MP_OK) cudaMemcpyAsync(host, c.flag, 2 * sizeof(int), cudaMemcpyDeviceToHost, s);
   const bool ok = cudaStreamSynchronize(s) == cudaSuccess && cudaGetLastError() == cudaSuccess;
-  if (c.buf) cudaFreeAsync(c.buf, s);
+  if (c.buf) scratch_free(c.buf, s);
   if (rc != MP_OK) return rc;
   if (!ok) return MP_ERR_CUDA;
   return host[1] ? MP_ERR_INVALID_ARG : MP_OK;
