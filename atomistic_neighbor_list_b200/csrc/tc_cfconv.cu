@@ -90,6 +90,7 @@ __global__ void __launch_bounds__(THREADS, 2) k_cfconv_fwd_tc(
   const int G = gridDim.x, cta = blockIdx.x;
 
   // ---- this CTA's destination rows: those whose first edge lies in [E c / G, E (c+1) / G)
+  E = clamp_off(row_ptr[N], E);  // the edges the list holds (E may be an upper bound of them)
   if (tid == 0) {
     const long long b_lo = E * cta / G, b_hi = E * (cta + 1) / G;
     const int r0 = lower_row(row_ptr, N, b_lo);

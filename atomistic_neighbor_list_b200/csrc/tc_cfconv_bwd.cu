@@ -89,6 +89,7 @@ __global__ void __launch_bounds__(THREADS, 2) k_cfconv_bwd_tc(
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, cta = blockIdx.x;
+  E = clamp_off(row_ptr[N], E);  // the edges the list holds (E may be an upper bound of them)
   if (tid == 0) {
     const long long b_lo = E * cta / G, b_hi = E * (cta + 1) / G;
     const int r0 = lower_row(row_ptr, N, b_lo);

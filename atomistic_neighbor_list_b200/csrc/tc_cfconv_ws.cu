@@ -118,6 +118,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_cfconv_fwd_ws(
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, cta = blockIdx.x;
+  E = clamp_off(row_ptr[N], E);  // the edges the list holds (E may be an upper bound of them)
   if (warp < 2) {  // this CTA's rows: an edge-balanced split, both ends searched at once
     const long long bnd = E * (cta + warp) / G;
     const int r = (warp == 1 && cta == G - 1) ? N : warp_lower_row(row_ptr, N, bnd);

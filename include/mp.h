@@ -261,7 +261,11 @@ int mp_set_graphs(mp_ctx* ctx, int on);
  *     units are the caller's, consistent with the energy unit and masses).
  *   The CSR (row_ptr, col_idx, graph_ptr) is NOT rebuilt: it must stay a superset of the pairs
  *     within r_c for all n_steps, e.g. built with cutoff r_c + skin and rebuilt by the caller
- *     before any atom has moved skin / 2 (pairs beyond r_c contribute exactly 0).
+ *     before any atom has moved skin / 2 (pairs beyond r_c contribute exactly 0). Each step first
+ *     cuts it to the pairs with d^2 < r_c^2 at that step's positions (fp32, each product and sum
+ *     rounded on its own, so the cut list stays symmetric) in scratch from the library's pool
+ *     (4 (N + 1) + 4 E bytes for the call), and runs the force kernels on the cut list: a skin
+ *     costs the cut, not force work on the pairs beyond r_c.
  *   kinetic: float32 [n_graphs] (device), or NULL: per-graph kinetic energy sum m_i |v_i|^2 / 2
  *     after the last step (fixed-order reduction).
  *   On a non-default stream with graphs on, the step is recorded once as a CUDA graph and
@@ -289,7 +293,8 @@ int mp_md_verlet(mp_ctx* ctx, int N, long long E, float* pos, float* vel, float*
  * check_every = 1 guarantees it.
  *   row_ptr int32 [N+1], col_idx int32 [capacity] (device): the list, owned by the caller;
  *   *n_edges (HOST) receives the edge count of the last build, *n_builds (HOST, or NULL) the
- *   number of builds. Other arguments as mp_md_verlet. Each check and each build synchronises
+ *   number of builds. Other arguments as mp_md_verlet (the force kernels run on the list cut to
+ *   r_c at each step's positions, as there). Each check and each build synchronises
  *   `stream`; steps between checks are replayed from one recorded CUDA graph per build.
  * Errors: MP_ERR_INVALID_ARG (non-finite dt, skin or max_disp, skin < 0, check_every < 1,
  * rebuild_every < 0), MP_ERR_CAPACITY (a list larger than capacity or the context's max_edges:

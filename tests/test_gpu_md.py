@@ -219,6 +219,36 @@ def test_md_no_atoms(mp):
 
 
 # ----------------------------------------------------------------------------- list maintenance
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_md_verlet_skin_list_costs_only_the_cut(mp, dtype):
+    """Each step cuts the list to the pairs within r_c before the force kernels: a list built at
+    r_c + 1 A and the exact r_c list give the same trajectory (the pairs between r_c and r_c + 1 A
+    have f_c = f_c' = 0; the two runs differ only where a pair crossed r_c during the steps, by
+    the rounding of a different tile partition). 3,000 atoms: many tiles on every CTA."""
+    wl = dataclasses.replace(synth.scaled(synth.WORKLOADS["cfg2"], 3000), dtype=dtype)
+    pos, _, types, im, v0 = md_inputs(wl, seed=3)
+    p0 = dev(pos)
+    rp_s, ci_s = mp.neighbor_csr(p0, wl.r_c + 1.0)
+    rp_x, ci_x = mp.neighbor_csr(p0, wl.r_c)
+    assert ci_s.numel() > 1.5 * ci_x.numel()
+    ctx = mp.Context.from_workload(wl, synth.make_weights(wl), max_atoms=len(pos),
+                                  max_edges=ci_s.numel())
+    runs = []
+    for rp, ci in ((rp_s, ci_s), (rp_x, ci_x)):
+        p, v, t = dev(pos), dev(v0), dev(types)
+        _, f = ctx.energy_forces(p, t, rp_x, ci_x)
+        f = f.clone()
+        e, _ = ctx.md_verlet(p, v, f, t, rp, ci, 4, 0.002, inv_mass=dev(im))
+        torch.cuda.synchronize()
+        ctx.status_sync()
+        runs.append((p.cpu().numpy(), f.cpu().numpy(), float(e[0])))
+    (ps, fs, es), (px, fx, ex) = runs
+    ftol, etol = (1e-5, 1e-6) if dtype == "fp32" else (5e-3, 1e-4)
+    assert np.abs(ps - px).max() <= 1e-5
+    assert rel_rms(fs, fx) <= ftol
+    assert abs(es - ex) <= etol * abs(ex)
+
+
 def fast_system(n=300, seed=5, vscale=1.5):
     """fp32, one interaction block; velocities large enough that atoms cross the rebuild limit."""
     wl = dataclasses.replace(synth.scaled(synth.WORKLOADS["cfg2"], n), dtype="fp32", n_blocks=1)
