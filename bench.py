@@ -480,7 +480,8 @@ def main():
         ms_md = sum(a.elapsed_time(b) for a, b in evm) / (len(evm) * md_steps)
         md = {"value": 1000.0 / ms_md, "unit": "MD steps/s", "ms_per_step": ms_md,
               "workload": f"{wl.name}: velocity Verlet, CSR at r_c + {skin} A skin "
-                          f"({ci_s.numel()} edges), {md_steps} steps per call, graph replay"}
+                          f"({ci_s.numel()} edges), {md_steps} steps per call, graph replay; "
+                          "each step cuts the list to r_c before the force kernels"}
         # the same loop maintaining its own list: rebuilt every 10 steps and whenever an atom
         # has moved 0.25 A (checked after every step), forces re-evaluated with each new list
         cap = 2 * ci_s.numel()
