@@ -106,9 +106,37 @@ __device__ __forceinline__ bool mbar_test(uint64_t* m, uint32_t parity) {
 }
 
 // Bounded wait on an mbarrier phase; false if the limit ran out.
+// try_wait with a suspend-time hint: a thread whose phase is not complete sleeps until it
+// completes or the hint (ns) expires, instead of returning at once to poll again.
+__device__ __forceinline__ bool mbar_try_sleep(uint64_t* m, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n.reg .pred P1;\nmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2, %3;\n"
+      "selp.b32 %0, 1, 0, P1;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(m)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+constexpr uint32_t kSuspendHintNs = 1000000;      // at most 1 ms asleep per try
+constexpr uint64_t kWaitBudgetNs = 2000000000ull;  // a wait gives up after 2 s
+
+// Wait for the phase of the given parity: at most `limit` tries and kWaitBudgetNs of global time,
+// whichever ends first. Returns false when it gave up (the caller reports a timeout).
 __device__ __forceinline__ bool mbar_wait(uint64_t* m, uint32_t parity, uint32_t limit) {
-  for (uint32_t i = 0; i < limit; ++i)
-    if (mbar_try(m, parity)) return true;
+  if (mbar_try_sleep(m, parity, kSuspendHintNs)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1; i < limit; ++i) {
+    if (mbar_try_sleep(m, parity, kSuspendHintNs)) return true;
+    if (global_ns() - t0 > kWaitBudgetNs) return false;
+  }
   return false;
 }
 
