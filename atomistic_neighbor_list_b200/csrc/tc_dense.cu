@@ -291,6 +291,13 @@ __global__ void __launch_bounds__(D2THREADS) k_dense2_tc(Dense2Args a, int* stat
       tc::commit(&mbar1);
     }
   }
+  // the residual this thread's 64 columns add to, requested before the wait for the first MMA
+  float4 old[16];
+  const bool resid = a.mode1 == MODE_RESIDUAL && valid;
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    old[i] = resid ? ((const float4*)(a.out1 + (size_t)r * 128 + 64 * half))[i]
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
   bool ok = !__syncthreads_or(bad);
   if (ok) {
     ok = !__syncthreads_or(tc::mbar_wait(&mbar1, 0, WAIT_LIMIT) ? 0 : 1);
@@ -298,8 +305,9 @@ __global__ void __launch_bounds__(D2THREADS) k_dense2_tc(Dense2Args a, int* stat
   }
   if (ok) {
     // ---- first layer's epilogue: the updated row, kept in fp32 and staged as bf16
-#pragma unroll 1
-    for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
+#pragma unroll
+    for (int hc = 0; hc < 2; ++hc) {
+      const int c0 = 64 * half + 32 * hc;
       uint32_t rr[32];
       tc::ld32(lane_base + c0, rr);
       tc::ld_wait();
@@ -308,17 +316,12 @@ __global__ void __launch_bounds__(D2THREADS) k_dense2_tc(Dense2Args a, int* stat
       for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(rr[i]) + (a.b1 ? a.b1[c0 + i] : 0.f);
       if (valid) {
         float4* o = (float4*)(a.out1 + (size_t)r * 128 + c0);
-        if (a.mode1 == MODE_RESIDUAL) {
-          float4 old[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) old[i] = o[i];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            v[4 * i] += old[i].x;
-            v[4 * i + 1] += old[i].y;
-            v[4 * i + 2] += old[i].z;
-            v[4 * i + 3] += old[i].w;
-          }
+        for (int i = 0; i < 8; ++i) {
+          v[4 * i] += old[8 * hc + i].x;
+          v[4 * i + 1] += old[8 * hc + i].y;
+          v[4 * i + 2] += old[8 * hc + i].z;
+          v[4 * i + 3] += old[8 * hc + i].w;
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
