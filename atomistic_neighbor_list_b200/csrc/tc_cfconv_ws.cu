@@ -384,7 +384,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_cfconv_fwd_ws(
       const int b = i & 1;
       if (!wait_warp(B_DONE1 + b, (i >> 1) & 1)) return false;
       tc::fence_after();
-      const float fc = MB(i % NMETA)->fc[e_me];
+      const float fc = MB(i % NMETA)->fc[e_me], fcln2 = fc * LN2;
       uint8_t* H = HB(b);
       uint32_t r[32];
       tc::ld32(lane_base + 128 * b + f0, r);
@@ -395,8 +395,8 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_cfconv_fwd_ws(
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int k = 8 * g8 + 2 * q;
-          w[q] = tc::pack_bf16(ssp_fc_poly(__uint_as_float(r[k]), fc),
-                               ssp_fc_poly(__uint_as_float(r[k + 1]), fc));
+          w[q] = tc::pack_bf16(ssp_scaled(__uint_as_float(r[k]), fc, fcln2),
+                               ssp_scaled(__uint_as_float(r[k + 1]), fc, fcln2));
         }
         *(uint4*)(H + kmaj(e_me, f0 + 8 * g8, K2)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
