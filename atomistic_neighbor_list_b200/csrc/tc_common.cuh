@@ -42,29 +42,6 @@ __device__ __forceinline__ float ssp_scaled(float z, float fc, float fcln2) {
   return fmaf(fcln2, l, fc * fmaxf(z, 0.f));
 }
 
-// ln((1 + t) / 2) on t in [0, 1]: degree-5 polynomial fitted here (Chebyshev least squares on
-// [0, 1]); absolute error below 1.1e-5, far under the bf16 rounding of the result.
-__device__ __forceinline__ float ln_half_one_plus(float t) {
-  float r = 0.030449004843831062f;
-  r = fmaf(r, t, -0.13158182799816132f);
-  r = fmaf(r, t, 0.2852726876735687f);
-  r = fmaf(r, t, -0.4902307093143463f);
-  r = fmaf(r, t, 0.9992355108261108f);
-  return fmaf(r, t, -0.6931372284889221f);
-}
-
-// 1 / (1 + t) on t in [0, 1]: degree-6 polynomial fitted here (Chebyshev least squares on
-// [0, 1]); absolute error below 7.5e-6.
-__device__ __forceinline__ float inv_one_plus(float t) {
-  float r = 0.07388167083263397f;
-  r = fmaf(r, t, -0.3292984962463379f);
-  r = fmaf(r, t, 0.6753469705581665f);
-  r = fmaf(r, t, -0.9070757627487183f);
-  r = fmaf(r, t, 0.9863784909248352f);
-  r = fmaf(r, t, -0.999220073223114f);
-  return fmaf(r, t, 0.9999925494194031f);
-}
-
 // Named barrier over n threads; the _or form also returns the OR of pred over them.
 __device__ __forceinline__ void bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -81,12 +58,6 @@ __device__ __forceinline__ bool bar_sync_or(int id, int n, bool pred) {
 }
 __device__ __forceinline__ void mbar_arrive1(uint64_t* m) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(tc::smem_u32(m)) : "memory");
-}
-
-// f_c * ssp(z) with one special-function op: ssp(z) = max(z, 0) + ln((1 + e^-|z|) / 2).
-__device__ __forceinline__ float ssp_fc_poly(float z, float fc) {
-  const float t = tc::ex2f(-fabsf(z) * LOG2E);
-  return fc * (fmaxf(z, 0.f) + ln_half_one_plus(t));
 }
 
 __device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
