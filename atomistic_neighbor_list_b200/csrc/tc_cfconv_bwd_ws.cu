@@ -590,9 +590,6 @@ __global__ void __launch_bounds__(BW_THREADS, 1) k_cfconv_bwd_ws(
         uint32_t w[4];
 #pragma unroll
         for (int p2 = 0; p2 < 4; ++p2) {
-          // g_k h_j + g_j h_k for two features in packed bf16 (rounded to bf16; the sum over the
-          // features below is fp32)
-          const uint32_t ap = tc::bfma2(a_gk[p2], a_hj[p2], tc::bmul2(a_gj[p2], a_hk[p2]));
           float m2[2];
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
@@ -601,9 +598,11 @@ __global__ void __launch_bounds__(BW_THREADS, 1) k_cfconv_bwd_ws(
             const float Wv = fc * U;
             const float Wp = fmaf(dfc, U, fc * __uint_as_float(cv[ii]));
             const float xgj = hh ? bf_hi(a_gj[p2]) : bf_lo(a_gj[p2]);
-            const float pa = hh ? bf_hi(ap) : bf_lo(ap);
+            const float xhj = hh ? bf_hi(a_hj[p2]) : bf_lo(a_hj[p2]);
+            const float xgk = hh ? bf_hi(a_gk[p2]) : bf_lo(a_gk[p2]);
+            const float xhk = hh ? bf_hi(a_hk[p2]) : bf_lo(a_hk[p2]);
             m2[hh] = xgj * Wv;
-            s_acc = fmaf(pa, Wp, s_acc);
+            s_acc = fmaf(fmaf(xgk, xhj, xgj * xhk), Wp, s_acc);
           }
           w[p2] = tc::pack_bf16(m2[0], m2[1]);
         }
