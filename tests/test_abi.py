@@ -61,6 +61,16 @@ def test_strerror_and_host_checks(lib):
     assert L.mp_neighbor_csr(-1, None, None, 1, 5.0, None, None, 0, None, None) == -1
     assert L.mp_neighbor_padded(4, None, None, 1, 5.0, 0, None, None, None) == -1
     assert L.mp_launch_count(None) == -1
+    # the later entry points: a null context or a bad size is rejected on the host
+    assert L.mp_attn_eq_fwd(None, 1, 1, None, None, None, None, None, None) == -1
+    assert L.mp_attn_bwd(None, 1, 1, None, None, None, None, None, None, None, None) == -1
+    assert L.mp_md_verlet(None, 1, 0, None, None, None, None, 0.01, 1, None, None, None, None, 1,
+                          None, None, None) == -1
+    n_edges = ctypes.c_longlong(0)
+    assert L.mp_md_run(None, 1, None, None, None, None, 0.01, 1, None, None, 1, 0.5, 10, 0.25, 1,
+                       None, None, 0, ctypes.byref(n_edges), None, None, None, None) == -1
+    assert L.mp_spatial_order(-1, None, None, 1, 5.0, None, None) == -1
+    assert L.mp_spatial_order(4, None, None, 1, 0.0, None, None) == -1
 
 
 def test_struct_layout_matches_header(lib):
