@@ -130,6 +130,9 @@ int mp_status_sync(mp_ctx* ctx, void* stream);
  * graph_ptr: int32 [n_graphs+1] contiguous atom ranges (device), or NULL for one graph.
  * Output: row_ptr [N+1], col_idx [capacity] (device), rows sorted by source index.
  * *n_edges (HOST pointer) receives E. Synchronises `stream` (to read E).
+ * Scratch: the cell grid and the sorted positions, O(N) bytes, stream-ordered from a memory pool
+ * the library keeps per device; the pool keeps what was freed for the next call (it holds at
+ * most the largest scratch live at once) instead of returning it at each synchronisation.
  * Errors: MP_ERR_INVALID_ARG, MP_ERR_CAPACITY (E > capacity; row_ptr is valid, col_idx not). */
 int mp_neighbor_csr(int N, const float* pos, const int* graph_ptr, int n_graphs, float r_c,
                     int* row_ptr, int* col_idx, long long capacity, long long* n_edges,
@@ -139,7 +142,8 @@ int mp_neighbor_csr(int N, const float* pos, const int* graph_ptr, int n_graphs,
  * skipped by a mask]. Same rule as mp_neighbor_csr; a row with more than K neighbors keeps the
  * K nearest by (d2, j); kept neighbors are stored by ascending j, then nbr = -1, mask = 0.
  * nbr int32 [N][K], mask uint8 [N][K] (device). A row with more than 1024 candidates raises
- * MP_ERR_CAPACITY (reported by the return value; synchronises `stream`).                      */
+ * MP_ERR_CAPACITY (reported by the return value; synchronises `stream`). Scratch as
+ * mp_neighbor_csr.                                                                            */
 int mp_neighbor_padded(int N, const float* pos, const int* graph_ptr, int n_graphs, float r_c,
                        int K, int* nbr, unsigned char* mask, void* stream);
 
@@ -150,7 +154,8 @@ int mp_neighbor_padded(int N, const float* pos, const int* graph_ptr, int n_grap
  * order; graphs keep their ranges, so graph_ptr stays valid for the permuted system. A caller
  * that applies the permutation to its per-atom arrays (positions, types, velocities, features)
  * gets the same physics with neighbors close in memory (the energy and forces are those of the
- * relabelled system). perm: int32 [N] (device). Synchronises `stream`.
+ * relabelled system). perm: int32 [N] (device). Synchronises `stream`. Scratch as
+ * mp_neighbor_csr.
  * Errors: MP_ERR_INVALID_ARG, MP_ERR_CAPACITY, MP_ERR_CUDA.                                    */
 int mp_spatial_order(int N, const float* pos, const int* graph_ptr, int n_graphs, float cell,
                      int* perm, void* stream);
@@ -197,7 +202,8 @@ int mp_attn_eq_fwd(mp_ctx* ctx, int N, int K, const float* pos, const int* nbr,
  * source-side position terms); deterministic. Needs n_heads * head_dim = F, n_heads <= 32,
  * head_dim dividing 32, and 16 K n_heads + 16 K bytes of per-row slot data on chip beside the
  * filter weights (K <= 256 at F = 128, n_rbf = 50, 16 heads), else MP_ERR_CAPACITY; N K < 2^31.
- * Allocates and frees O(N K) bytes of stream-ordered scratch (the transposed list).
+ * Allocates and frees O(N K) bytes of stream-ordered scratch (the transposed list) from the
+ * library's per-device pool (as mp_neighbor_csr).
  * Errors: MP_ERR_INVALID_ARG, MP_ERR_CAPACITY, MP_ERR_CUDA.                                    */
 int mp_attn_bwd(mp_ctx* ctx, int N, int K, const float* pos, const int* nbr,
                 const unsigned char* mask, const void* x, const float* g_out, float* grad_x,
