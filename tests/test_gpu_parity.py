@@ -1,7 +1,10 @@
 """CUDA path vs the fp64 oracle, through the C-ABI, on seeded inputs of the five workloads.
 
 Neighbor lists and indices are compared bit for bit. Features: normwise max|d|/max|ref| <= 1e-5 on
-the fp32 path and <= 2e-2 on the bf16 path; forces: relative RMS <= 1e-2 on the bf16 path. The bf16
+the fp32 path and <= 2e-2 on the bf16 path; forces: relative RMS <= 1e-2 on the bf16 path and
+<= 1e-4 on the fp32 path (no stated bound; derived: an atom's force is the sum of its pair terms
+over the blocks, whose absolute sum is 4-6 times the net force on these systems, so the fp32
+feature bound 1e-5 becomes ~6e-5 on the net force, rounded up to 1e-4). The bf16
 oracle is the same fp64 code fed the bf16-rounded inputs and weights the library holds, so only the
 CUDA path's own intermediate roundings are measured. Full-size workloads are compared on sampled
 rows the oracle computes one by one, and through properties that hold at any size.
