@@ -81,6 +81,8 @@ def test_md_verlet_matches_oracle(mp, dtype, n):
     r, v, fr, er = oracle.velocity_verlet(run.oracle_force, run.pos, run.v0, f0, dt, steps, run.im)
     got_r, got_v, got_f = (t.cpu().numpy().astype(np.float64) for t in (pos, vel, f))
     assert np.abs(r - run.pos).max() < SKIN / 2
+    # forces and velocities at the force bounds; positions: coordinates up to ~20 A are stored in
+    # fp32 (ulp 2e-6 A), so 2e-5 A is ten ulps (fp32) and 2e-4 A leaves room for the bf16 forces
     ftol = 1e-4 if dtype == "fp32" else TOL_BF16_FORCE
     assert np.abs(got_r - r).max() <= (2e-5 if dtype == "fp32" else 2e-4)
     assert rel_rms(got_v, v) <= ftol
@@ -283,6 +285,9 @@ def test_md_run_matches_fresh_exact_lists(mp):
     got = p.cpu().numpy().astype(np.float64)
     assert np.abs(r - pos).max() > 2 * skin  # far enough that the list had to be rebuilt
     assert out["n_builds"] >= 3
+    # 40 fp32 steps at high velocity: the fp32 rounding of each step grows along the trajectory
+    # (and the two sides cut their lists at different moments), so 1e-3 instead of the one-step
+    # bounds
     assert np.abs(got - r).max() <= 1e-3
     assert rel_rms(v.cpu().numpy(), vr) <= 1e-3
     assert rel_rms(out["forces"].cpu().numpy(), fr) <= 1e-3
