@@ -337,6 +337,88 @@ def test_exact_zero_at_cutoff():
     assert abs(E2[0] - E[0]) < 1e-4
 
 
+# ----------------------------------------------------------------------------- energy forward by hand
+def _hand_ssp(v: float) -> float:
+    return math.log(0.5 * math.exp(v) + 0.5)
+
+
+def _hand_readout(w, x):
+    """e = ssp(x B1 + d1) B2 + d2 with plain Python loops (x: list of F floats)."""
+    B1, d1, B2, d2 = (np.asarray(w[k], dtype=float) for k in ("B1", "d1", "B2", "d2"))
+    F, Fh = B1.shape
+    e = float(d2[0])
+    for g in range(Fh):
+        a = float(d1[g]) + sum(x[f] * float(B1[f, g]) for f in range(F))
+        e += _hand_ssp(a) * float(B2[g, 0])
+    return e
+
+
+def _hand_dense(W, b, x):
+    W, b = np.asarray(W, dtype=float), np.asarray(b, dtype=float)
+    return [float(b[o]) + sum(x[i] * float(W[i, o]) for i in range(len(x))) for o in range(W.shape[1])]
+
+
+def test_isolated_atom_energy_by_hand():
+    # no neighbor: m = 0 in every block, so x_B = emb[t] + sum_b b_out_b and
+    # E = ssp((emb[t] + sum_b b_out_b) B1 + d1) B2 + d2 -- pins the embedding row, the residual
+    # bias of every block and every readout term (a dropped b_out, d1, d2 or a wrong type row fails)
+    model, w, wl = small_model(F=6, R=5, n_blocks=3, n_types=4)
+    for t in range(4):
+        pos = np.array([[1.0, 2.0, 3.0]], dtype=np.float32)
+        types = np.array([t], dtype=np.int32)
+        rp, ci = oracle.neighbor_csr(pos, 5.0)
+        x = [float(v) for v in w["emb"][t]]
+        for b in range(3):
+            x = [x[f] + float(w[f"b_out.{b}"][f]) for f in range(6)]
+        want = _hand_readout(w, x)
+        got = oracle.energies(model, pos, types, rp, ci)[0]
+        assert abs(got - want) <= 1e-12 * max(1.0, abs(want)), (t, got, want)
+    # far-apart atoms: the energy is the sum of the isolated atoms' energies
+    pos = np.array([[0, 0, 0], [50, 0, 0], [0, 50, 0], [0, 0, 50]], dtype=np.float32)
+    types = np.array([3, 0, 2, 0], dtype=np.int32)
+    rp, ci = oracle.neighbor_csr(pos, 5.0)
+    singles = []
+    for t in types:
+        x = [float(v) for v in w["emb"][t]]
+        for b in range(3):
+            x = [x[f] + float(w[f"b_out.{b}"][f]) for f in range(6)]
+        singles.append(_hand_readout(w, x))
+    assert abs(oracle.energies(model, pos, types, rp, ci)[0] - sum(singles)) <= 1e-12 * 4
+
+
+@pytest.mark.parametrize("n_blocks", [1, 2])
+def test_two_atom_energy_by_hand(n_blocks):
+    # every stage of the forward written out with math for a bound pair: embedding, per block
+    # h = x W_in + b_in, m_i = h_j (.) W(d), x <- x + m W_out + b_out, then the readout of both atoms
+    F, R = 4, 5
+    model, w, wl = small_model(F=F, R=R, n_blocks=n_blocks, n_types=3)
+    pos = np.array([[0.3, -0.2, 0.1], [2.1, 1.4, -1.9]], dtype=np.float32)
+    types = np.array([2, 0], dtype=np.int32)
+    rp, ci = oracle.neighbor_csr(pos, 5.0)
+    assert ci.tolist() == [1, 0]
+    p = pos.astype(float)
+    d = math.sqrt(sum((p[0, c] - p[1, c]) ** 2 for c in range(3)))
+    mu = [5.0 * k / (R - 1) for k in range(R)]
+    e = [math.exp(-10.0 * (d - mu[k]) ** 2) for k in range(R)]
+    fc = 0.5 * (math.cos(math.pi * d / 5.0) + 1.0)
+    xs = [[float(v) for v in w["emb"][t]] for t in types]
+    for b in range(n_blocks):
+        A1, c1, A2, c2 = (np.asarray(w[f"{k}.{b}"], dtype=float) for k in ("A1", "c1", "A2", "c2"))
+        h1 = [_hand_ssp(sum(e[k] * A1[k, g] for k in range(R)) + c1[g]) for g in range(F)]
+        Wd = [fc * (sum(h1[g] * A2[g, f] for g in range(F)) + c2[f]) for f in range(F)]
+        hs = [_hand_dense(w[f"W_in.{b}"], w[f"b_in.{b}"], x) for x in xs]
+        ms = [[hs[1][f] * Wd[f] for f in range(F)], [hs[0][f] * Wd[f] for f in range(F)]]
+        outs = [_hand_dense(w[f"W_out.{b}"], w[f"b_out.{b}"], m) for m in ms]
+        xs = [[xs[a][f] + outs[a][f] for f in range(F)] for a in range(2)]
+    want = _hand_readout(w, xs[0]) + _hand_readout(w, xs[1])
+    got = oracle.energies(model, pos, types, rp, ci)[0]
+    assert abs(got - want) <= 1e-12 * max(1.0, abs(want)), (got, want)
+    # the same number from energy_forces (both force forms) and per-atom energies by hand
+    E_s, _, e_atom = oracle.energy_forces(model, pos, types, rp, ci, return_atom_energy=True)
+    assert abs(E_s[0] - want) <= 1e-12 * max(1.0, abs(want))
+    assert abs(e_atom[0] - _hand_readout(w, xs[0])) <= 1e-12 * max(1.0, abs(e_atom[0]))
+
+
 # ----------------------------------------------------------------------------- attention
 def test_attention_uniform_weights_give_mean():
     model, w, wl = small_model(F=8, n_heads=2, head_dim=4)
