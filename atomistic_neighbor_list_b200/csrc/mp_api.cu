@@ -282,6 +282,16 @@ extern "C" int mp_status_sync(mp_ctx* c, void* stream) {
 
 extern "C" long long mp_launch_count(mp_ctx* c) { return c ? c->launches : -1; }
 
+extern "C" int mp_set_wait_budget(mp_ctx* c, long long ns) {
+  if (!c || ns < 0) return MP_ERR_INVALID_ARG;
+  c->wait_ns = (unsigned long long)ns;
+  if (c->ef_graph) {  // the budget is a kernel argument: a recorded graph holds the old one
+    cudaGraphExecDestroy(c->ef_graph);
+    c->ef_graph = nullptr;
+  }
+  return MP_OK;
+}
+
 // ---------------------------------------------------------------------------------------------
 extern "C" int mp_cfconv_fwd(mp_ctx* c, int block, int N, long long E, const float* pos,
                              const int* row_ptr, const int* col_idx, const void* x, void* out,

@@ -79,6 +79,8 @@ struct mp_ctx {
   int* md_flag = nullptr;                 // status_d + 1: an atom moved past the rebuild limit
   int* md_flag_h = nullptr;               // status_h + 1
   long long launches = 0;
+  // budget of every bounded device wait in the tensor-core kernels (ns of global time)
+  unsigned long long wait_ns = 2000000000ull;
   // CUDA graph of the last energy/forces call, replayed when a call repeats its arguments
   bool graphs = true, graphs_broken = false;
   cudaGraphExec_t ef_graph = nullptr;

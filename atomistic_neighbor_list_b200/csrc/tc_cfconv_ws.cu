@@ -97,7 +97,8 @@ template <int K1>
 __global__ void __launch_bounds__(WS_THREADS, 1) k_cfconv_fwd_ws(
     int N, long long E, const float* __restrict__ pos, const int* __restrict__ row_ptr,
     const int* __restrict__ col_idx, const __nv_bfloat16* __restrict__ x,
-    __nv_bfloat16* __restrict__ out, const uint8_t* __restrict__ img, Radial rp, int* status) {
+    __nv_bfloat16* __restrict__ out, const uint8_t* __restrict__ img, Radial rp, int* status,
+    unsigned long long wait_ns) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   constexpr WsSmem L = ws_layout(K1);
@@ -161,7 +162,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_cfconv_fwd_ws(
   const uint32_t tmem = *s_tmem;
   volatile int* abort_flag = &s_misc[10];
   auto wait_bar = [&](int idx, uint32_t parity) -> bool {
-    if (tc::mbar_wait(&bars[idx], parity, WAIT_LIMIT)) return true;
+    if (tc::mbar_wait_ns(&bars[idx], parity, WAIT_LIMIT, wait_ns)) return true;
     *abort_flag = 1;
     return false;
   };
@@ -512,6 +513,8 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_cfconv_fwd_ws(
       zero_rows(out, next_row, r_end, e_me);
     }
   }
+  // the weight copy has landed before the CTA exits, whatever the roles gave up on (full budget)
+  if (tid == 0) tc::mbar_wait(&bars[B_W], 0, WAIT_LIMIT);
   tc::fence_before();
   __syncthreads();
   if (tid == 0 && *abort_flag) raise_status(status, kStatusTimeout);
@@ -537,7 +540,7 @@ int tc_cfconv_fwd_ws(mp_ctx* ctx, int block, int N, long long E, const float* po
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     return launch(ctx, K_CFCONV_FWD_TC, kern, dim3(grid), dim3(WS_THREADS), smem, s, N, E, pos,
                   row_ptr, col_idx, (const __nv_bfloat16*)x, (__nv_bfloat16*)out, img, radial_of(ctx),
-                  ctx->status_d);
+                  ctx->status_d, (unsigned long long)ctx->wait_ns);
   };
   static_assert(ws_fits(64) && ws_fits(48) && ws_fits(32) && !ws_fits(80), "shared memory plan");
   if (K1 == 64) return go(k_cfconv_fwd_ws<64>, 64);

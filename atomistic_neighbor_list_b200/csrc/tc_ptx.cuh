@@ -140,6 +140,21 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* m, uint32_t parity, uint32_t
   return false;
 }
 
+// The same wait with a caller-given budget of global time (ns) instead of kWaitBudgetNs: one
+// quick test, then suspend-hinted tries until the phase completes or the budget has passed
+// (at most `limit` tries). A zero budget gives up at once unless the phase is already complete.
+__device__ __forceinline__ bool mbar_wait_ns(uint64_t* m, uint32_t parity, uint32_t limit,
+                                             uint64_t budget_ns) {
+  if (mbar_try(m, parity)) return true;
+  if (budget_ns == 0) return false;
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 0; i < limit; ++i) {
+    if (mbar_try_sleep(m, parity, kSuspendHintNs)) return true;
+    if (global_ns() - t0 >= budget_ns) return false;
+  }
+  return false;
+}
+
 // Expect `bytes` of asynchronous (TMA) traffic on the mbarrier and arrive once.
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* m, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(m)),
@@ -154,18 +169,6 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
           smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(m))
-      : "memory");
-}
-
-// TMA row gather: rows r0..r3 of a 2-D tensor map (columns c0 .. c0 + box width) into four
-// consecutive box rows of this CTA's shared memory, completing on an mbarrier. The map's box is one
-// row high; c0 times the element size is a multiple of 16 bytes. No multicast.
-__device__ __forceinline__ void tma_gather4(void* dst, const void* tmap, int c0, int r0, int r1,
-                                            int r2, int r3, uint64_t* m) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
-      "l"(tmap), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(m))
       : "memory");
 }
 
@@ -245,6 +248,16 @@ __device__ __forceinline__ void ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
+}
+
+// 32 lanes x 32 bits, 4 consecutive columns stored from this thread's registers (its lane).
+__device__ __forceinline__ void st4(uint32_t taddr, const uint32_t (&r)[4]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
+               : "memory");
+}
+__device__ __forceinline__ void st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {

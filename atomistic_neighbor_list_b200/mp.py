@@ -65,6 +65,7 @@ def _load():
         "mp_profile_end": (i32, [vp, vp]),
         "mp_profile_get": (i32, [vp, i32, POINTER(c_char_p), POINTER(c_double), POINTER(i64)]),
         "mp_launch_count": (i64, [vp]),
+        "mp_set_wait_budget": (i32, [vp, i64]),
         "mp_set_graphs": (i32, [vp, i32]),
         "mp_md_verlet": (i32, [vp, i32, i64, vp, vp, vp, vp, c_float, i32, vp, vp, vp, vp, i32,
                                vp, vp, vp]),
@@ -90,7 +91,8 @@ EXPORTED = ("mp_init", "mp_destroy", "mp_strerror", "mp_status_sync", "mp_neighb
             "mp_neighbor_padded", "mp_cfconv_fwd", "mp_attn_fwd", "mp_energy_forces",
             "mp_profile_begin", "mp_profile_end", "mp_profile_get", "mp_launch_count",
             "mp_attn_fwd_noalloc", "mp_selftest_tc", "mp_set_graphs",
-            "mp_md_verlet", "mp_md_run", "mp_attn_bwd", "mp_attn_eq_fwd", "mp_spatial_order")
+            "mp_md_verlet", "mp_md_run", "mp_attn_bwd", "mp_attn_eq_fwd", "mp_spatial_order",
+            "mp_set_wait_budget")
 NOALLOC_MAX_NF = 524288  # MP_NOALLOC_MAX_NF: largest N * F mp_attn_fwd_noalloc accepts
 
 
@@ -275,6 +277,10 @@ class Context:
     def launch_count(self) -> int:
         return int(lib.mp_launch_count(self._ctx))
 
+    def set_wait_budget(self, ns: int):
+        """mp_set_wait_budget: give up every bounded device wait after ns nanoseconds."""
+        _check(lib.mp_set_wait_budget(self._ctx, int(ns)), "mp_set_wait_budget")
+
     def md_verlet(self, pos, vel, forces, types, row_ptr, col_idx, n_steps, dt, inv_mass=None,
                   graph_ptr=None, energy=None, kinetic=None, stream=None):
         """mp_md_verlet: n_steps velocity-Verlet steps in place on pos, vel, forces (forces must
@@ -388,12 +394,19 @@ def attn_fwd_noalloc(*, F: int, n_rbf: int, n_heads: int, head_dim: int, r_c: fl
     cfg = MpConfig(F=F, n_rbf=n_rbf, n_blocks=1, n_types=1, n_heads=n_heads, head_dim=head_dim,
                    r_c=r_c, gamma=gamma, mu_min=mu_min, mu_max=r_c if mu_max is None else mu_max,
                    dtype=FP32, max_atoms=N, max_edges=0, max_graphs=1, validate=0)
+    # the C entry point reads F*F floats of Wq, Wk and A2, n_rbf*F of A1, n_rbf*n_heads of P: a
+    # short or misplaced array would be read past its end, so the shapes and the device are checked
+    shapes = {"Wq": (F, F), "Wk": (F, F), "P": (n_rbf, n_heads), "p": (n_heads,),
+              "A1.0": (n_rbf, F), "c1.0": (F,), "A2.0": (F, F), "c2.0": (F,)}
+    for key, shape in shapes.items():
+        t = _need(weights[key], key, torch.float32, shape)
+        if t.device != x.device:
+            raise ValueError(f"{key}: must be on {x.device}, got {t.device}")
     w = MpWeights()
     for key in ("Wq", "Wk", "P", "p"):
-        setattr(w, key, ctypes.cast(_need(weights[key], key, torch.float32).data_ptr(), _FP))
+        setattr(w, key, ctypes.cast(weights[key].data_ptr(), _FP))
     for key in ("A1", "c1", "A2", "c2"):
-        getattr(w, key)[0] = ctypes.cast(_need(weights[f"{key}.0"], key, torch.float32).data_ptr(),
-                                         _FP)
+        getattr(w, key)[0] = ctypes.cast(weights[f"{key}.0"].data_ptr(), _FP)
     w.on_device = 1
     _check(lib.mp_attn_fwd_noalloc(ctypes.byref(cfg), ctypes.byref(w), N, K, _ptr(pos), _ptr(nbr),
                                    _ptr(mask), _ptr(x), _ptr(out), _ptr(status), _stream(stream)),

@@ -40,6 +40,8 @@ def parse():
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--workload", default="cfg2")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--configs", default="cfg1,cfg3,cfg4,cfg5",
+                    help="other workloads measured beside the main line (comma list; empty: none)")
     ap.add_argument("--profile-run", action="store_true",
                     help="short run for ncu: no clocks sampler, no e2e, no CPU baseline")
     return ap.parse_args()
@@ -148,9 +150,10 @@ def gpu_uuid(torch, dev):
 
 # ------------------------------------------------------------------------------ work model
 def kernel_model(name: str, wl, E: int, N: int):
-    """(bound, algorithmic FLOPs or bytes per launch, unit) for a library kernel."""
+    """(bound, algorithmic FLOPs or bytes per launch, unit) for a library kernel. E is the number
+    of edges one launch processes (valid edges for the attention)."""
     R, F = wl.n_rbf, wl.F
-    fwd = 2.0 * (R * F + F * F) * E
+    fwd = 2.0 * (R * F + F * F) * E  # filter MLP per edge: R -> F, then F -> F
     if name == "cfconv_fwd_simt":
         return "alu", fwd, "TFLOP/s"
     if name == "cfconv_bwd_simt":
@@ -159,9 +162,45 @@ def kernel_model(name: str, wl, E: int, N: int):
         return "tensor", fwd, "TFLOP/s"
     if name == "cfconv_bwd_tc":
         return "tensor", 2.0 * fwd, "TFLOP/s"
+    if name == "attn_tc":  # filter MLP + per-head radial logit bias + q.k per valid edge
+        return "tensor", fwd + 2.0 * (R * wl.n_heads + F) * E, "TFLOP/s"
     if name == "dense":
         return "hbm", (4 + 2 + 4) * N * F, "GB/s"
     return "hbm", 0.0, "GB/s"
+
+
+def peak_for(bound: str, peaks: dict, clocks):
+    """Roofline denominator and its source. Tensor-bound kernels are timed here in regions well
+    under a second: the burst bf16 peak applies unless the sampled clocks show the power-capped
+    state the sustained figure was measured in (sw_power_cap with the SM clock below 90 % of max)."""
+    src = peaks["source"]
+    if bound == "tensor":
+        capped = bool(clocks) and "sw_power_cap" in clocks.get("reasons", []) and \
+            clocks.get("sm_mhz", 0) < 0.9 * clocks.get("sm_max_mhz", 1)
+        if capped:
+            return peaks["bf16_tflops_sustained"], f"{src} bf16 sustained (power-capped clocks seen)"
+        return peaks["bf16_tflops"], f"{src} bf16 burst (clocks at max, sub-second timed regions)"
+    if bound == "alu":
+        return (148 * FP32_LANES_PER_SM * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12,
+                "FP32 FMA: 148 SMs x 128 lanes x 2 flop x max SM clock")
+    return peaks["hbm_gbs"], f"{src} HBM copy"
+
+
+def roofline_of(prof: dict, wl, E: int, N: int, peaks: dict, clocks, per_unit_ms=None):
+    """The dominant kernel of a profiled run against its roofline."""
+    if not prof:
+        return None
+    name, st = max(prof.items(), key=lambda kv: kv[1]["total_ms"])
+    avg_ms = st["total_ms"] / st["launches"]
+    bound, work, unit = kernel_model(name, wl, E, N)
+    peak, note = peak_for(bound, peaks, clocks)
+    achieved = work / (avg_ms / 1000.0) / (1e12 if unit == "TFLOP/s" else 1e9)
+    out = {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+           "frac": achieved / peak, "avg_launch_ms": avg_ms, "launches": st["launches"],
+           "peak_source": note, "work_per_launch": work}
+    if per_unit_ms:
+        out["share_of_step"] = st["total_ms"] / per_unit_ms
+    return out
 
 
 KERNEL_SOURCES = {  # the files whose contents decide a kernel's traffic
@@ -217,6 +256,190 @@ def cpu_baseline(wl, full_edges: int, budget_s: float):
             "sample": f"one energy+forces step of a {n}-atom same-density system ({e1} edges, "
                       f"{t1:.2f} s), scaled to the {full_edges}-edge workload by edge count",
             "seconds": t1}
+
+
+def _host_cores():
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+
+
+def cpu_legs(key: str, full_units: float, budget_s: float = 3.0):
+    """The fp64 oracle, as it stands, timed single-threaded and on all host cores on a bounded
+    sample of one workload; each leg is scaled to the workload's own unit (edges/s of a block,
+    valid edges/s of the attention, or energy+forces steps/s of the whole system). The sample is
+    chosen so that one leg takes about ``budget_s`` of CPU time on one thread."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    import oracle
+    from atomistic_neighbor_list_b200 import synth
+    wl = synth.WORKLOADS["cfg2" if key == "cfg2_block" else key]
+    model = oracle.Model.from_workload(wl, synth.make_weights(wl))
+
+    if key in ("cfg1", "cfg2_block"):
+        wl = synth.WORKLOADS["cfg1" if key == "cfg1" else "cfg2"]
+        model = oracle.Model.from_workload(wl, synth.make_weights(wl))
+        pos, _ = synth.positions_for(wl)
+        rp, ci = oracle.neighbor_csr(pos, wl.r_c)
+        x = synth.node_features(len(pos), wl.F)
+
+        def run(frac):  # the first rows of the workload, about frac of its edges
+            n = max(1, int(len(pos) * frac))
+            rows = np.arange(n)
+            t = time.perf_counter()
+            oracle.cfconv(model, 0, pos, rp, ci, x, rows=rows)
+            return time.perf_counter() - t, int(rp[n] - rp[0]), f"{n} of {len(pos)} rows"
+        unit, scale_kind = "edges/s", "edges"
+    elif key == "cfg4":
+        pos, _ = synth.positions_for(wl)
+        nbr, mask = oracle.neighbor_padded(pos, wl.r_c, wl.K)
+        x = synth.node_features(len(pos), wl.F)
+
+        def run(frac):
+            n = max(1, int(len(pos) * frac))
+            rows = np.arange(n)
+            t = time.perf_counter()
+            oracle.attention(model, pos, nbr, mask, x, rows=rows)
+            return time.perf_counter() - t, int(mask[:n].sum()), f"{n} of {len(pos)} rows"
+        unit, scale_kind = "edges/s", "valid edges"
+    elif key == "cfg3":
+        beads = wl.n_atoms // wl.replicas
+
+        def run(frac):  # k of the 64 independent replicas: the work scales exactly with k
+            k = max(1, int(round(wl.replicas * frac)))
+            pos, gp = synth.chain_replicas(k, beads, seed=0)
+            types = synth.atom_types(len(pos), wl.n_types)
+            rp, ci = oracle.neighbor_csr(pos, wl.r_c, gp)
+            t = time.perf_counter()
+            oracle.energy_forces(model, pos, types, rp, ci, gp)
+            return time.perf_counter() - t, k / wl.replicas, f"{k} of {wl.replicas} replicas"
+        unit, scale_kind = UNIT, "replicas"
+    else:  # cfg2 / cfg5 energy + forces: a same-density smaller system, scaled by edge count
+        def run(frac):
+            n = max(64, int(wl.n_atoms * frac))
+            sw = synth.scaled(wl, n)
+            pos, _ = synth.positions_for(sw)
+            types = synth.atom_types(n, wl.n_types)
+            rp, ci = oracle.neighbor_csr(pos, wl.r_c)
+            t = time.perf_counter()
+            oracle.energy_forces(model, pos, types, rp, ci)
+            return time.perf_counter() - t, len(ci), f"a {n}-atom same-density system"
+        unit, scale_kind = UNIT, "edges"
+
+    # calibration sample: a few hundred atoms (rows, one replica), then one sized to the budget
+    frac0 = {"cfg1": 1.0, "cfg3": 1.0 / wl.replicas}.get(key, min(1.0, 300.0 / wl.n_atoms))
+
+    def leg(threads):
+        with threadpool_limits(threads):
+            t1, u1, what = run(frac0)
+            frac = min(1.0, frac0 * budget_s / max(t1, 1e-3) * 0.8)
+            if frac > 1.5 * frac0:
+                t1, u1, what = run(frac)
+        if unit == UNIT:  # whole-system steps/s: the sample did u1 of the work of one step
+            share = u1 if scale_kind == "replicas" else u1 / full_units
+            value = share / t1
+        else:
+            value = u1 / t1
+        return {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
+                "sample": f"{what} ({t1:.2f} s), scaled by {scale_kind}"}
+
+    return {"single_thread": leg(1), "all_cores": leg(_host_cores())}
+
+
+def measure_configs(keys, devn, stream, flush, steps: int):
+    """Throughput of the other workloads on this GPU, each with the same timing rules as the main
+    line (CUDA events on the launching stream, L2 flushed between timed calls, warm-up first,
+    atoms in cell order). Returns {key: result} plus the per-kernel profiles for the rooflines."""
+    import numpy as np
+    import torch
+
+    from atomistic_neighbor_list_b200 import mp, synth
+    out, profs = {}, {}
+
+    def timed(fn, n):
+        evs = []
+        for _ in range(n):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            evs.append((a, b))
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in evs) / n
+
+    def profiled(ctx, fn, n):
+        ctx.profile_begin()
+        for _ in range(n):
+            flush.zero_()
+            fn()
+        return ctx.profile_end()
+
+    def system(wl):
+        pos, gp = synth.positions_for(wl)
+        G = len(gp) - 1
+        gp_d = torch.from_numpy(gp).to(devn) if G > 1 else None
+        perm = mp.spatial_order(torch.from_numpy(pos).to(devn), wl.r_c, graph_ptr=gp_d)
+        perm = perm.cpu().numpy()
+        pos = np.ascontiguousarray(pos[perm])
+        types = np.ascontiguousarray(synth.atom_types(len(pos), wl.n_types)[perm])
+        pos_d = torch.from_numpy(pos).to(devn)
+        rp, ci = mp.neighbor_csr(pos_d, wl.r_c, graph_ptr=gp_d)
+        return pos_d, torch.from_numpy(types).to(devn), gp_d, G, rp, ci
+
+    n_calls = max(10, steps)
+    for key in keys:
+        wl = synth.WORKLOADS[key]
+        if key == "cfg4":
+            pos, _ = synth.positions_for(wl)
+            pos_d = torch.from_numpy(pos).to(devn)
+            nbr, mask = mp.neighbor_padded(pos_d, wl.r_c, wl.K)
+            valid = int(mask.sum().item())
+            ctx = mp.Context.from_workload(wl, synth.make_weights(wl), max_atoms=len(pos),
+                                           max_edges=1)
+            x = torch.from_numpy(synth.node_features(len(pos), wl.F)).to(devn).to(torch.bfloat16)
+            o = torch.empty_like(x)
+            fn = lambda: ctx.attn_fwd(pos_d, nbr, mask, x, o)
+            for _ in range(3):
+                fn()
+            ms = timed(fn, max(10, steps // 3))
+            profs[key] = (profiled(ctx, fn, 5), wl, valid, len(pos), ms)
+            ctx.status_sync()
+            out[key] = {"workload": wl.name, "atoms": len(pos), "valid_edges": valid,
+                        "K": wl.K, "dtype": wl.dtype, "edges_per_s": valid / (ms / 1000.0),
+                        "ms_per_call": ms, "call": "mp_attn_fwd (q/k projections included)"}
+            ctx.close()
+            continue
+        pos_d, types_d, gp_d, G, rp, ci = system(wl)
+        E, N = ci.numel(), pos_d.shape[0]
+        ctx = mp.Context.from_workload(wl, synth.make_weights(wl), max_atoms=N, max_edges=E,
+                                       max_graphs=G)
+        tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+        x = torch.from_numpy(synth.node_features(N, wl.F)).to(devn).to(tdt)
+        m = torch.empty_like(x)
+        blk = lambda: ctx.cfconv_fwd(0, pos_d, rp, ci, x, m)
+        for _ in range(3):
+            blk()
+        ms_blk = timed(blk, n_calls)
+        res = {"workload": wl.name, "atoms": N, "edges": E, "dtype": wl.dtype,
+               "block_edges_per_s": E / (ms_blk / 1000.0), "ms_per_block": ms_blk}
+        if wl.kind == "cfconv":
+            profs[key] = (profiled(ctx, blk, 5), wl, E, N, ms_blk)
+        else:
+            energy = torch.empty(G, dtype=torch.float32, device=devn)
+            forces = torch.empty((N, 3), dtype=torch.float32, device=devn)
+            ef = lambda: ctx.energy_forces(pos_d, types_d, rp, ci, gp_d, energy, forces)
+            for _ in range(3):
+                ef()
+            ms = timed(ef, n_calls)
+            res.update({"steps_per_s": 1000.0 / ms, "ms_per_step": ms, "graphs": G,
+                        "launch": "energy_forces replayed from one recorded CUDA graph"})
+            if G > 1:  # FlashSchNet's unit: timesteps x molecules per second
+                res["timestep_mol_per_s"] = G * 1000.0 / ms
+            profs[key] = (profiled(ctx, ef, 5), wl, E, N, ms)
+        ctx.status_sync()
+        out[key] = res
+        ctx.close()
+    return out, profs
 
 
 def reference_arm(args):
@@ -319,10 +542,9 @@ def main():
 
     clocks = None
     if not args.profile_run:
-        clocks = Clocks(gpu_uuid(torch, local), os.path.join(ROOT, "gpurun_out",
-                                                               f"clocks_rank{rank}.csv")
-                        if os.path.isdir(os.path.join(ROOT, "gpurun_out"))
-                        else f"/tmp/mp_clocks_{os.getpid()}.csv")
+        import tempfile
+        clocks = Clocks(gpu_uuid(torch, local),
+                        os.path.join(tempfile.gettempdir(), f"mp_clocks_{os.getpid()}_{rank}.csv"))
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -560,39 +782,35 @@ def main():
         bo = h_energy.numel() * 4 + h_forces.numel() * 4
         e2e = {"value": job_value(world, args.steps, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo)}
+    configs, cprofs = {}, {}
+    if not args.profile_run and rank == 0 and args.configs:
+        configs, cprofs = measure_configs([k for k in args.configs.split(",") if k], devn, stream,
+                                          flush, args.steps)
     ck = clocks.stop() if clocks else None
     ctx.status_sync()
 
     # ---- roofline of the dominant kernel (from the timed region's per-kernel events)
-    roofline = None
+    roofline = roofline_of(prof, wl, E, N, peaks, ck, per_unit_ms=total_ms)
     kernels = {}
-    if prof:
-        top = max(prof.items(), key=lambda kv: kv[1]["total_ms"])
-        name, st = top
-        avg_ms = st["total_ms"] / st["launches"]
-        bound, work, unit = kernel_model(name, wl, E, N)
-        if bound == "tensor":
-            peak = peaks["bf16_tflops_sustained"]
-            peak_note = f"{peaks['source']} bf16 sustained"
-        elif bound == "alu":
-            peak = 148 * FP32_LANES_PER_SM * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
-            peak_note = "FP32 FMA: 148 SMs x 128 lanes x 2 flop x max SM clock"
-        else:
-            peak = peaks["hbm_gbs"]
-            peak_note = f"{peaks['source']} HBM copy"
-        achieved = work / (avg_ms / 1000.0) / (1e12 if unit == "TFLOP/s" else 1e9)
-        traffic = traffic_for(name, E)
-        roofline = {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak,
-                    "unit": unit, "frac": achieved / peak, "traffic": traffic,
-                    "avg_launch_ms": avg_ms, "launches": st["launches"],
-                    "share_of_step": st["total_ms"] / max(total_ms, 1e-9),
-                    "peak_source": peak_note}
+    if roofline:
+        roofline["traffic"] = traffic_for(roofline["kernel"], E)
         kernels = {k: {"ms_per_step": v["total_ms"] / args.steps,
                        "launches_per_step": v["launches"] / args.steps} for k, v in prof.items()}
+    for key, (p, cwl, units, n_at, ms) in cprofs.items():
+        rl = roofline_of(p, cwl, units, n_at, peaks, ck)
+        if rl:
+            rl["share_of_call"] = p[rl["kernel"]]["total_ms"] / sum(v["total_ms"] for v in p.values())
+        configs[key]["roofline"] = rl
 
     cpu = None
+    cpu_extra = {}
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile_run:
         cpu = cpu_baseline(wl, E, budget_s=15.0)
+        cpu_extra["cfg2_energy_forces"] = cpu_legs("cfg2", E)
+        cpu_extra["cfg2_block"] = cpu_legs("cfg2_block", E)
+        for key, res in configs.items():
+            units = res.get("edges", res.get("valid_edges"))
+            res["cpu_baseline"] = cpu_legs(key, units)
 
     if rank == 0:
         res = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -609,7 +827,10 @@ def main():
                "attention_edges_per_s": attn,
                "md_loop": md,
                "edges_per_s_per_block": {"value": edges_per_s, "unit": "edges/s",
-                                         "ms_per_block": cf_total},
+                                         "ms_per_block": cf_total,
+                                         "cpu_baseline": cpu_extra.get("cfg2_block")},
+               "cpu_legs": cpu_extra.get("cfg2_energy_forces"),
+               "configs": configs,
                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
                "clocks": ck, "kernels": kernels}
         print(json.dumps(res), flush=True)

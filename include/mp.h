@@ -323,6 +323,19 @@ int mp_profile_get(mp_ctx* ctx, int index, const char** name, double* total_ms,
 /* Number of kernels this context has launched since mp_init.                               */
 long long mp_launch_count(mp_ctx* ctx);
 
+/* Budget of the bounded device waits (a library addition, no counterpart on the pages). The
+ * warp-specialised tensor-core kernels hand tiles between their warp roles through shared-memory
+ * barriers; every such wait gives up after `ns` nanoseconds of GPU global time (default
+ * 2,000,000,000), after which the kernel stops its roles in order (each MMA-issuing thread still
+ * waits, with the default budget, for everything it issued), frees its tensor memory, returns
+ * normally and raises MP_ERR_TIMEOUT, read by the next mp_status_sync; outputs are then
+ * unspecified. A small budget makes waits run out on purpose (a test of that path); 0 gives up
+ * unless the awaited phase is already complete. Later calls of the context use the new budget
+ * (a recorded energy/forces graph is dropped, since it holds the old one). Applies to the cfconv
+ * forward and backward kernels of the bf16 path.
+ * Errors: MP_ERR_INVALID_ARG (ns < 0).                                                       */
+int mp_set_wait_budget(mp_ctx* ctx, long long ns);
+
 /* Diagnostic: run the tensor-core layout self-check on the current device (one CTA; exact small-
  * integer products through the shared-memory operand layouts the kernels use). mismatches (HOST,
  * int[2]) receives the number of wrong outputs of the two checks (0 = pass; negative = an MMA did

@@ -83,7 +83,7 @@ def test_md_verlet_matches_oracle(mp, dtype, n):
     assert np.abs(r - run.pos).max() < SKIN / 2
     # forces and velocities at the force bounds; positions: coordinates up to ~20 A are stored in
     # fp32 (ulp 2e-6 A), so 2e-5 A is ten ulps (fp32) and 2e-4 A leaves room for the bf16 forces
-    ftol = 1e-4 if dtype == "fp32" else TOL_BF16_FORCE
+    ftol = 1e-5 if dtype == "fp32" else TOL_BF16_FORCE
     assert np.abs(got_r - r).max() <= (2e-5 if dtype == "fp32" else 2e-4)
     assert rel_rms(got_v, v) <= ftol
     assert rel_rms(got_f, fr) <= ftol

@@ -2,9 +2,8 @@
 
 Neighbor lists and indices are compared bit for bit. Features: normwise max|d|/max|ref| <= 1e-5 on
 the fp32 path and <= 2e-2 on the bf16 path; forces: relative RMS <= 1e-2 on the bf16 path and
-<= 1e-4 on the fp32 path (no stated bound; derived: an atom's force is the sum of its pair terms
-over the blocks, whose absolute sum is 4-6 times the net force on these systems, so the fp32
-feature bound 1e-5 becomes ~6e-5 on the net force, rounded up to 1e-4). The bf16
+<= 1e-5 on the fp32 path (the fp32 relative-error bound applied to the forces; measured on a B200:
+7e-7 to 8.4e-7 on the 64-, 300-, 700- and 2,000-atom systems, energies 4e-8 to 2e-7). The bf16
 oracle is the same fp64 code fed the bf16-rounded inputs and weights the library holds, so only the
 CUDA path's own intermediate roundings are measured. Full-size workloads are compared on sampled
 rows the oracle computes one by one, and through properties that hold at any size.
@@ -309,8 +308,8 @@ def ef_case(mp, key, n=None, dtype=None, seed=0):
 def test_energy_forces_fp32(mp, key, n):
     wl_key = key
     E, F, Eref, Fref, scale = ef_case(mp, wl_key, n=n, dtype="fp32")
-    assert np.max(np.abs(E - Eref) / scale) <= 1e-5
-    assert rel_rms(F, Fref) <= 1e-4
+    assert np.max(np.abs(E - Eref) / scale) <= TOL_FP32
+    assert rel_rms(F, Fref) <= TOL_FP32
 
 
 @pytest.mark.parametrize("key,n", [("fd64", 64), ("cfg2", 10_000)])

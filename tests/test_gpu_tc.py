@@ -159,3 +159,37 @@ def test_forces_sixty_four_radial_functions(mp):
     pos, _ = synth.chain_replicas(3, 250, seed=2)
     e_err, f_err, tol = run_ef(mp, pos, r_c=10.0, n_rbf=64)
     assert e_err <= TOL_BF16_FEAT and f_err <= tol
+
+
+# ----------------------------------------------------------------------------- bounded waits
+def test_bounded_wait_timeout_is_reported_and_the_context_recovers(mp):
+    """The warp-specialised cfconv kernels hand tiles between warp roles through shared-memory
+    barriers, every wait bounded by the context's budget. With a zero budget the waits give up at
+    once: the kernels stop their roles in order, free their tensor memory and return, and the
+    status word reports MP_ERR_TIMEOUT (no trap, no fault, no hang). With the default budget
+    restored the next call on the same context matches the oracle."""
+    from helpers import TOL_BF16_FORCE, rel_rms
+    wl = synth.scaled(synth.WORKLOADS["cfg2"], 400)
+    pos = synth.uniform_positions(400, seed=21)
+    types = synth.atom_types(400, wl.n_types, seed=22)
+    w = synth.make_weights(wl)
+    pos_d = torch.from_numpy(pos).cuda()
+    types_d = torch.from_numpy(types).cuda()
+    rp, ci = mp.neighbor_csr(pos_d, wl.r_c)
+    ctx = mp.Context.from_workload(wl, w, max_atoms=400, max_edges=ci.numel())
+    ctx.set_wait_budget(0)
+    for _ in range(2):  # both cfconv directions run; a second call finds a clean context too
+        ctx.energy_forces(pos_d, types_d, rp, ci)
+        torch.cuda.synchronize()
+        with pytest.raises(mp.MpError) as e:
+            ctx.status_sync()
+        assert e.value.name == "MP_ERR_TIMEOUT"
+    ctx.set_wait_budget(2_000_000_000)
+    E, F = ctx.energy_forces(pos_d, types_d, rp, ci)
+    torch.cuda.synchronize()
+    ctx.status_sync()
+    model = oracle.Model.from_workload(wl, oracle_weights(w, "bf16"))
+    orp, oci = oracle_csr(pos, wl.r_c, rp, ci)
+    Eref, Fref, e_atom = oracle.energy_forces(model, pos, types, orp, oci, return_atom_energy=True)
+    assert abs(float(E[0]) - Eref[0]) / np.abs(e_atom).sum() <= TOL_BF16_FEAT
+    assert rel_rms(F.cpu().numpy(), Fref) <= TOL_BF16_FORCE
