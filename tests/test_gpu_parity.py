@@ -326,33 +326,40 @@ def test_energy_forces_bf16_replicas(mp):
     assert rel_rms(F, Fref) <= TOL_BF16_FORCE
 
 
-def test_energy_forces_full_100k_properties(mp):
-    """100k atoms: net force ~ 0 and sampled forces vs the oracle on a cut-out sphere.
-
-    A force on atom k depends only on atoms within 2 * n_blocks * r_c of it, so the oracle on the
-    atoms within that radius (plus a margin) of a sampled atom gives that atom's exact force.
-    """
+def test_energy_forces_full_100k_against_the_oracle(mp):
+    """100,000 atoms (the full workload) in the launch configuration the bench times: atoms
+    relabelled in cell order, energy_forces recorded as a CUDA graph on a side stream and replayed.
+    Compared with the fp64 oracle's energy and all 100,000 forces of the same system, which
+    tests/golden/make_cfg5_oracle.py stored (it calls only the oracle; about ten minutes of CPU):
+    energy within 2e-2 of the sum of |atomic energies|, forces at relative RMS <= 1e-2."""
+    import hashlib
+    import os
+    g = np.load(os.path.join(os.path.dirname(__file__), "golden", "cfg5_oracle.npz"))
     wl = synth.WORKLOADS["cfg5"]
     pos, _ = synth.positions_for(wl)
     n = len(pos)
     types = synth.atom_types(n, wl.n_types)
-    w = synth.make_weights(wl)
-    rp, ci = mp.neighbor_csr(dev(pos), wl.r_c)
-    ctx, _ = make_ctx(mp, wl, w, n, ci.numel())
-    E, F = ctx.energy_forces(dev(pos), dev(types), rp, ci)
-    torch.cuda.synchronize()
-    ctx.status_sync()
-    F = F.cpu().numpy().astype(np.float64)
-    assert np.all(np.isfinite(F)) and np.isfinite(E.item())
+    h = hashlib.sha256()
+    h.update(np.ascontiguousarray(pos, dtype=np.float32).tobytes())
+    h.update(np.ascontiguousarray(types, dtype=np.int32).tobytes())
+    assert h.hexdigest()[:16] == str(g["digest"][0]), "the stored oracle values are of another system"
+    perm = mp.spatial_order(dev(pos), wl.r_c).cpu().numpy()
+    pos_p, types_p = np.ascontiguousarray(pos[perm]), np.ascontiguousarray(types[perm])
+    pos_d = dev(pos_p)
+    rp, ci = mp.neighbor_csr(pos_d, wl.r_c)
+    assert ci.numel() == int(g["edges"][0])
+    ctx, _ = make_ctx(mp, wl, synth.make_weights(wl), n, ci.numel())
+    stream = torch.cuda.Stream()
+    energy = torch.empty(1, dtype=torch.float32, device=DEV)
+    forces = torch.empty((n, 3), dtype=torch.float32, device=DEV)
+    with torch.cuda.stream(stream):
+        for _ in range(2):  # records the graph, then replays it
+            ctx.energy_forces(pos_d, dev(types_p), rp, ci, None, energy, forces, stream=stream)
+    stream.synchronize()
+    ctx.status_sync(stream)
+    F = np.empty((n, 3))
+    F[perm] = forces.cpu().numpy().astype(np.float64)
+    E = float(energy.item())
+    assert abs(E - float(g["energy"][0])) <= TOL_BF16_FEAT * float(g["energy_scale"][0])
+    assert rel_rms(F, g["forces"].astype(np.float64)) <= TOL_BF16_FORCE
     assert np.linalg.norm(F.sum(axis=0)) <= 1e-4 * np.linalg.norm(F, axis=1).sum()
-    centre = pos.mean(axis=0)
-    k = int(np.argmin(np.linalg.norm(pos - centre, axis=1)))
-    radius = 2 * wl.n_blocks * wl.r_c + 1.0
-    sel = np.nonzero(np.linalg.norm(pos - pos[k], axis=1) < radius)[0]
-    sub = pos[sel]
-    orp, oci = oracle.neighbor_csr(sub, wl.r_c)
-    model = oracle.Model.from_workload(wl, oracle_weights(w, wl.dtype))
-    _, Fsub = oracle.energy_forces(model, sub, types[sel], orp, oci)
-    kk = int(np.nonzero(sel == k)[0][0])
-    ref = Fsub[kk]
-    assert np.linalg.norm(F[k] - ref) <= 3e-2 * np.linalg.norm(ref)
