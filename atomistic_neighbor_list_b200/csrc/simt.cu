@@ -13,7 +13,7 @@
 namespace mp {
 
 constexpr int EB = 16;     // edges per batch
-constexpr int ROWS = 16;   // destination rows per CTA work item
+constexpr int ROWS = 16;   // destination rows per CTA work item (at most; small systems take fewer)
 
 FilterW filter_of(const mp_ctx* ctx, int b) {
   return FilterW{ctx->A1[b], ctx->c1[b], ctx->A2[b], ctx->c2[b]};
@@ -27,6 +27,14 @@ Radial radial_of(const mp_ctx* ctx) {
   r.dmu = (ctx->cfg.mu_max - ctx->cfg.mu_min) / (float)(ctx->cfg.n_rbf - 1);
   r.r_c = ctx->cfg.r_c;
   return r;
+}
+
+// Destination rows per CTA work item of the fp32 cfconv kernels: up to ROWS, fewer when that would
+// leave SMs idle (a 512-atom system in 16-row items is 32 CTAs of F threads on 148 SMs).
+static int rows_for(const mp_ctx* ctx, int N, int ctas_per_sm) {
+  const long long slots = (long long)ctx->num_sms * ctas_per_sm;
+  const long long r = (N + slots - 1) / slots;
+  return (int)(r < 1 ? 1 : (r > ROWS ? ROWS : r));
 }
 
 static int grid_for(const mp_ctx* ctx, long long items, int per_cta_items, int ctas_per_sm) {
@@ -201,7 +209,7 @@ template <typename T, int F>
 __global__ void __launch_bounds__(F) k_cfconv_fwd_simt(
     int N, long long E, const float* __restrict__ pos, const int* __restrict__ row_ptr,
     const int* __restrict__ col_idx, const T* __restrict__ x, T* __restrict__ out, FilterW fw,
-    Radial rp, int* status) {
+    Radial rp, int* status, int rows) {
   extern __shared__ float dsm[];
   float* sA1 = dsm;                 // [R][F]
   float* sA2 = dsm + rp.R * F;      // [F][F]
@@ -216,8 +224,8 @@ __global__ void __launch_bounds__(F) k_cfconv_fwd_simt(
   const float c1f = fw.c1[f], c2f = fw.c2[f];
   __syncthreads();
 
-  for (int r0 = blockIdx.x * ROWS; r0 < N; r0 += gridDim.x * ROWS) {
-    const int r1 = min(r0 + ROWS, N);
+  for (int r0 = blockIdx.x * rows; r0 < N; r0 += gridDim.x * rows) {
+    const int r1 = min(r0 + rows, N);
     const long long e_beg = clamp_off(row_ptr[r0], E);
     long long e_end = clamp_off(row_ptr[r1], E);
     if (e_end < e_beg) e_end = e_beg;
@@ -306,9 +314,11 @@ static int run_fwd(mp_ctx* ctx, int block, int N, long long E, const float* pos,
   size_t smem = (size_t)(R * F + F * F) * sizeof(float);
   auto kern = k_cfconv_fwd_simt<T, F>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  int grid = grid_for(ctx, N, ROWS, 2);
+  const int per_sm = F == 64 ? 4 : 2;  // CTAs one SM holds (shared memory)
+  const int rows = rows_for(ctx, N, per_sm);
+  int grid = grid_for(ctx, N, rows, per_sm);
   return launch(ctx, K_CFCONV_FWD_SIMT, kern, dim3(grid), dim3(F), smem, s, N, E, pos, rp, ci,
-                (const T*)x, (T*)out, filter_of(ctx, block), radial_of(ctx), ctx->status_d);
+                (const T*)x, (T*)out, filter_of(ctx, block), radial_of(ctx), ctx->status_d, rows);
 }
 
 int launch_cfconv_fwd_simt(mp_ctx* ctx, int block, int N, long long E, const float* pos,
@@ -334,7 +344,7 @@ __global__ void __launch_bounds__(F) k_cfconv_bwd_simt(
     int N, long long E, const float* __restrict__ pos, const int* __restrict__ row_ptr,
     const int* __restrict__ col_idx, const T* __restrict__ h, const T* __restrict__ g,
     float* __restrict__ grad_h, float* __restrict__ forces, int accumulate, FilterW fw, Radial rp,
-    int* status) {
+    int* status, int rows) {
   extern __shared__ float dsm[];
   float* sA1 = dsm;
   float* sA2 = dsm + rp.R * F;
@@ -351,8 +361,8 @@ __global__ void __launch_bounds__(F) k_cfconv_bwd_simt(
   const float c1f = fw.c1[f], c2f = fw.c2[f];
   __syncthreads();
 
-  for (int r0 = blockIdx.x * ROWS; r0 < N; r0 += gridDim.x * ROWS) {
-    const int r1 = min(r0 + ROWS, N);
+  for (int r0 = blockIdx.x * rows; r0 < N; r0 += gridDim.x * rows) {
+    const int r1 = min(r0 + rows, N);
     const long long e_beg = clamp_off(row_ptr[r0], E);
     long long e_end = clamp_off(row_ptr[r1], E);
     if (e_end < e_beg) e_end = e_beg;
@@ -514,10 +524,12 @@ static int run_bwd(mp_ctx* ctx, int block, int N, long long E, const float* pos,
   size_t smem = (size_t)(R * F + F * F) * sizeof(float);
   auto kern = k_cfconv_bwd_simt<T, F>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  int grid = grid_for(ctx, N, ROWS, 2);
+  const int per_sm = F == 64 ? 3 : 1;  // CTAs one SM holds (shared memory)
+  const int rows = rows_for(ctx, N, per_sm);
+  int grid = grid_for(ctx, N, rows, per_sm);
   return launch(ctx, K_CFCONV_BWD_SIMT, kern, dim3(grid), dim3(F), smem, s, N, E, pos, rp, ci,
                 (const T*)h, (const T*)g, grad_h, forces, (int)acc, filter_of(ctx, block),
-                radial_of(ctx), ctx->status_d);
+                radial_of(ctx), ctx->status_d, rows);
 }
 
 int launch_cfconv_bwd_simt(mp_ctx* ctx, int block, int N, long long E, const float* pos,

@@ -560,13 +560,23 @@ __global__ void __launch_bounds__(BW_THREADS, 1) k_cfconv_bwd_ws(
       const uint32_t zb = lane_base + f0;
       // the group's operand buffer holds msg^T of its previous tile until that segment sum is done
       if (i >= NGRP && !wait_warp(B_DONE3 + g, ((i - NGRP) >> 1) & 1)) return false;
+      // eight columns of z1 and of t per pass, the next pass's requested before this one is used
+      uint32_t rz[8], rt[8];
+      tc::ld8(zb, rz);
+      tc::ld8(zb + 128, rt);
 #pragma unroll
       for (int c = 0; c < FPT / 8; ++c) {
-        // eight columns of z1 and of t per pass (the other group's warps cover the load latency)
+        tc::ld_wait(rz, rt);
         uint32_t cz[8], ct[8];
-        tc::ld8(zb + 8 * c, cz);
-        tc::ld8(zb + 128 + 8 * c, ct);
-        tc::ld_wait(cz, ct);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          cz[k] = rz[k];
+          ct[k] = rt[k];
+        }
+        if (c + 1 < FPT / 8) {
+          tc::ld8(zb + 8 * (c + 1), rz);
+          tc::ld8(zb + 128 + 8 * (c + 1), rt);
+        }
         uint32_t wq[4], wp[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -627,6 +637,12 @@ __global__ void __launch_bounds__(BW_THREADS, 1) k_cfconv_bwd_ws(
       tc::fence_after();
       float sa = 0.f, sb = 0.f;
       const uint32_t ub = lane_base + f0;
+      // u, v eight columns per TMEM load, the next pass's requested before this one is used (a
+      // load waited for at once costs its whole latency, several hundred cycles while the tensor
+      // core works on the other group's tile)
+      uint32_t ru[8], rv[8];
+      tc::ld8(ub, ru);
+      tc::ld8(ub + 128, rv);
       // ---- sweep A: msg = g_j W -> QP (MN-major), sa += g_j h_k W'
 #pragma unroll
       for (int p = 0; p < FPT / 8; ++p) {
@@ -634,10 +650,18 @@ __global__ void __launch_bounds__(BW_THREADS, 1) k_cfconv_bwd_ws(
         const uint4 vgj = row[p], vhk = nhk;
         row[p] = __ldg(hj4 + p);
         if (p + 1 < FPT / 8) nhk = __ldg(hk4 + p + 1);
+        tc::ld_wait(ru, rv);
         uint32_t cu[8], cv[8];
-        tc::ld8(ub + 8 * p, cu);
-        tc::ld8(ub + 128 + 8 * p, cv);
-        tc::ld_wait(cu, cv);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          cu[k] = ru[k];
+          cv[k] = rv[k];
+        }
+        {  // the next pass (sweep B starts over at column 0)
+          const int pn = p + 1 < FPT / 8 ? p + 1 : 0;
+          tc::ld8(ub + 8 * pn, ru);
+          tc::ld8(ub + 128 + 8 * pn, rv);
+        }
         const uint32_t a_gj[4] = {vgj.x, vgj.y, vgj.z, vgj.w};
         const uint32_t a_hk[4] = {vhk.x, vhk.y, vhk.z, vhk.w};
         const float4 ca = *(const float4*)(sc2 + f8);
@@ -670,10 +694,17 @@ __global__ void __launch_bounds__(BW_THREADS, 1) k_cfconv_bwd_ws(
         const int f8 = f0 + 8 * p;
         const uint4 vhj = row[p], vgk = ngk;
         if (p + 1 < FPT / 8) ngk = __ldg(gk4 + p + 1);
+        tc::ld_wait(ru, rv);
         uint32_t cu[8], cv[8];
-        tc::ld8(ub + 8 * p, cu);
-        tc::ld8(ub + 128 + 8 * p, cv);
-        tc::ld_wait(cu, cv);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          cu[k] = ru[k];
+          cv[k] = rv[k];
+        }
+        if (p + 1 < FPT / 8) {
+          tc::ld8(ub + 8 * (p + 1), ru);
+          tc::ld8(ub + 128 + 8 * (p + 1), rv);
+        }
         const uint32_t a_hj[4] = {vhj.x, vhj.y, vhj.z, vhj.w};
         const uint32_t a_gk[4] = {vgk.x, vgk.y, vgk.z, vgk.w};
         const float4 ca = *(const float4*)(sc2 + f8);
