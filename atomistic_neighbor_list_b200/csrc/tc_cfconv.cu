@@ -497,7 +497,7 @@ int tc_cfconv_fwd_sequential(mp_ctx* ctx, int block, int N, long long E, const f
   auto go = [&](auto kern, int k1) {
     const size_t smem = smem_layout(k1).total + 1024;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    return launch(ctx, K_CFCONV_FWD_TC, kern, dim3(grid), dim3(THREADS), smem, s, N, E, pos,
+    return launch(ctx, K_CFCONV_FWD_TC_LS, kern, dim3(grid), dim3(THREADS), smem, s, N, E, pos,
                   row_ptr, col_idx, (const __nv_bfloat16*)x, (__nv_bfloat16*)out, img,
                   radial_of(ctx), ctx->status_d);
   };

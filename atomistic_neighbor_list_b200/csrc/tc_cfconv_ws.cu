@@ -13,8 +13,8 @@
 //                          every hand-off is an mbarrier (one arrival per warp)
 //   MMA1 (warp 20)         MMA1 of each tile once its Gaussian operand is written
 //   MMA2/3 (warp 21)       MMA2 and MMA3 in the order the epilogue produces their operands
-// Two TMEM accumulators of 128 columns and two Gaussian / h' operand buffers alternate between
-// tiles; the 0/1 matrix and the x_j rows have one buffer each. Every wait is bounded; a warp that
+// Two TMEM accumulators of 128 columns and two Gaussian (one for 64 radial functions) and two h'
+// operand buffers alternate between tiles; the 0/1 matrix and the x_j rows have one buffer each. Every wait is bounded; a warp that
 // gives up votes so within the warp, and the other roles then run out their own bounded waits.
 #include "tc_common.cuh"
 
@@ -40,6 +40,10 @@ struct WsMeta {
 struct WsSmem {
   uint32_t w1, w2, c2, a0, s, h0, x, meta0, rp, misc, bars, total;
 };
+// Gaussian operand buffers: two (the prep runs two tiles ahead) where they fit beside the staged
+// x_j rows, one for the wider operand of 64 radial functions (K1 = 80; the prep then runs one
+// tile ahead)
+__host__ __device__ constexpr int ws_nbuf_a(int K1) { return K1 <= 64 ? 2 : 1; }
 __host__ __device__ constexpr WsSmem ws_layout(int K1) {
   // W1, W2, c2 | Gaussian operand x2 | 0/1 matrix | h' / msg^T x2 | x_j rows | metadata x4 |
   // prep | misc | mbarriers
@@ -48,7 +52,7 @@ __host__ __device__ constexpr WsSmem ws_layout(int K1) {
   L.w1 = o;    o += FT * K1 * 2;
   L.w2 = o;    o += FT * K2 * 2;
   L.c2 = o;    o += 1024;
-  L.a0 = o;    o += 2 * TM * K1 * 2;
+  L.a0 = o;    o += ws_nbuf_a(K1) * TM * K1 * 2;
   L.s = o;     o += SMAX * TM * 2;
   L.h0 = o;    o += 2 * TM * K2 * 2;
   L.x = o;     o += TM * FT * 2;
@@ -102,6 +106,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_cfconv_fwd_ws(
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   constexpr WsSmem L = ws_layout(K1);
+  constexpr int NA = ws_nbuf_a(K1);
   uint8_t* sW1 = sm + L.w1;
   uint8_t* sW2 = sm + L.w2;
   float* sc2 = (float*)(sm + L.c2);
@@ -203,9 +208,10 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_cfconv_fwd_ws(
       const float pjx = pos[3 * j], pjy = pos[3 * j + 1], pjz = pos[3 * j + 2];
       const int wr = min(r_lo + t, N - 1);  // the window's rows hold this tile's destinations
       const float wx = pos[3 * wr], wy = pos[3 * wr + 1], wz = pos[3 * wr + 2];
-      // Gaussian operand buffer b is free once MMA1 of tile it-2 completed (and with it the
-      // metadata slot of tile it-4: its drain preceded that MMA1)
-      const bool free_ok = it < 2 || wait_bar(B_DONE1 + b, ((it - 2) >> 1) & 1);
+      // Gaussian operand buffer it % NA is free once MMA1 of tile it - NA completed (and with it
+      // the metadata slot of tile it-4: its drain preceded that MMA1)
+      const bool free_ok =
+          it < NA || wait_bar(B_DONE1 + ((it - NA) & 1), ((it - NA) >> 1) & 1);
       if (bar_sync_or(1, 128, !free_ok || *abort_flag)) {  // uniform over the prep warps
         live = false;
         break;
@@ -257,7 +263,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_cfconv_fwd_ws(
       s_pdst[t] = my_dst;
       // Gaussian operand row (bf16), bias column R = 1, zero padding
       const float d0 = d - rp.mu_min;
-      uint8_t* A = AB(b);
+      uint8_t* A = AB(it % NA);
 #pragma unroll
       for (int k0 = 0; k0 < K1; k0 += 8) {
         uint32_t w[4];
@@ -313,7 +319,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_cfconv_fwd_ws(
       if (!ok) break;
       tc::fence_after();
       if (lane == 0) {
-        const uint32_t sA_a = tc::smem_u32(AB(b));
+        const uint32_t sA_a = tc::smem_u32(AB(n % NA));
         for (int ks = 0; ks < K1 / 16; ++ks)
           tc::mma(tmem + 128 * b, tc::sdesc(sA_a + ks * 256, 128, K1 * 16),
                   tc::sdesc(sW1_a + ks * 256, 128, K1 * 16), id12, ks > 0);
@@ -529,7 +535,7 @@ int tc_cfconv_fwd_ws(mp_ctx* ctx, int block, int N, long long E, const float* po
   const int K1 = k1_of(ctx->cfg.n_rbf);
   const ImgLayout IL = img_layout(K1);
   const uint8_t* img = (const uint8_t*)ctx->tc_weights + IL.bytes * block;
-  // 64 < n_rbf < 80: the staged x_j rows no longer fit beside the wider Gaussian operand
+  // a Gaussian operand wider than the shared-memory plan allows: the lock-step kernel
   if (!ws_fits(K1))
     return tc_cfconv_fwd_sequential(ctx, block, N, E, pos, row_ptr, col_idx, x, out, s);
   long long tiles = (E + TM - 1) / TM;
@@ -542,7 +548,8 @@ int tc_cfconv_fwd_ws(mp_ctx* ctx, int block, int N, long long E, const float* po
                   row_ptr, col_idx, (const __nv_bfloat16*)x, (__nv_bfloat16*)out, img, radial_of(ctx),
                   ctx->status_d, (unsigned long long)ctx->wait_ns);
   };
-  static_assert(ws_fits(64) && ws_fits(48) && ws_fits(32) && !ws_fits(80), "shared memory plan");
+  static_assert(ws_fits(80) && ws_fits(64) && ws_fits(48) && ws_fits(32), "shared memory plan");
+  if (K1 == 80) return go(k_cfconv_fwd_ws<80>, 80);
   if (K1 == 64) return go(k_cfconv_fwd_ws<64>, 64);
   if (K1 == 48) return go(k_cfconv_fwd_ws<48>, 48);
   if (K1 == 32) return go(k_cfconv_fwd_ws<32>, 32);

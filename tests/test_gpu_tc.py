@@ -193,3 +193,23 @@ def test_bounded_wait_timeout_is_reported_and_the_context_recovers(mp):
     Eref, Fref, e_atom = oracle.energy_forces(model, pos, types, orp, oci, return_atom_energy=True)
     assert abs(float(E[0]) - Eref[0]) / np.abs(e_atom).sum() <= TOL_BF16_FEAT
     assert rel_rms(F.cpu().numpy(), Fref) <= TOL_BF16_FORCE
+
+
+def test_sixty_four_radial_functions_run_warp_specialised(mp):
+    """The chain workload's 64 radial functions (a 16-bit Gaussian operand of 80 columns) run on
+    the warp-specialised forward and backward kernels, not on the lock-step fallbacks."""
+    wl = synth.WORKLOADS["cfg3"]
+    pos, gp = synth.chain_replicas(4, 200, seed=3)
+    n = len(pos)
+    pos_d = torch.from_numpy(pos).cuda()
+    gp_d = torch.from_numpy(gp).cuda()
+    rp, ci = mp.neighbor_csr(pos_d, wl.r_c, graph_ptr=gp_d)
+    ctx = mp.Context.from_workload(wl, synth.make_weights(wl), max_atoms=n, max_edges=ci.numel(),
+                                   max_graphs=4)
+    types = torch.from_numpy(synth.atom_types(n, wl.n_types)).cuda()
+    ctx.profile_begin()
+    ctx.energy_forces(pos_d, types, rp, ci, gp_d)
+    prof = ctx.profile_end()
+    ctx.status_sync()
+    assert "cfconv_fwd_tc" in prof and "cfconv_bwd_tc" in prof, prof
+    assert not any(k.endswith("_lockstep") for k in prof), prof
