@@ -221,7 +221,8 @@ extern "C" int mp_init(mp_ctx** out_ctx, const mp_config* cfg, const mp_weights*
                     nf * 4,            // grad_h
                     nf * 4, nf * 4,    // q, k
                     N * 3 * 4,         // md_ref
-                    N * 3 * (size_t)(H > 0 ? H : 1) * 4};  // attn_stats
+                    N * 3 * (size_t)(H > 0 ? H : 1) * 4,   // attn_stats
+                    (N / 1024 + (size_t)cfg->max_graphs + 8) * 4};  // gsum_part
   size_t ws = 0;
   for (size_t v : sizes) ws += align_up(v, 256);
   char* wsb = nullptr;
@@ -249,6 +250,7 @@ extern "C" int mp_init(mp_ctx** out_ctx, const mp_config* cfg, const mp_weights*
   c->k = (float*)take(sizes[10]);
   c->md_ref = (float*)take(sizes[11]);
   c->attn_stats = (float*)take(sizes[12]);
+  c->gsum_part = (float*)take(sizes[13]);
   if (cudaMalloc(&c->status_d, 4 * sizeof(int)) != cudaSuccess ||
       cudaMallocHost(&c->status_h, 4 * sizeof(int)) != cudaSuccess) {
     free_ctx(c);

@@ -67,6 +67,7 @@ struct mp_ctx {
   float* a = nullptr;                     // [N][F/2] readout pre-activation
   float* u_ro = nullptr;                  // [N][F/2] readout backward
   float* e_atom = nullptr;                // [N]
+  float* gsum_part = nullptr;             // per-graph energy partials: N / 1024 + max_graphs
   float* g_x = nullptr;                   // [N][F] dE/dx
   void* g_m = nullptr;                    // [N][F] storage dtype: dE/dm
   float* grad_h = nullptr;                // [N][F] dE/dh
