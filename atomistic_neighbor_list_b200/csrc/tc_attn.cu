@@ -161,7 +161,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1) k_attn_tc(
   if (warp < PREP_WARPS) {
     // =============================================================== prep role (128 threads)
     const int t = tid;
-    const float nglog2e = -rp.gamma * LOG2E;
+    const float xs = sqrtf(rp.gamma * LOG2E), dmu_x = rp.dmu * xs;
+    const float rstep = tc::ex2f(-2.f * dmu_x * dmu_x), pi_rc = 3.14159265358979f / rp.r_c;
     // the x_j rows of tile k, once every epilogue warp has read those of tile k-1 (16 threads per
     // 256-byte row); false on abort, uniformly over the prep warps
     auto gather = [&](int k) -> bool {
@@ -210,7 +211,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1) k_attn_tc(
       if (ok) {
         const float dx = pix - pjx, dy = piy - pjy, dz = piz - pjz;
         d = sqrtf(dx * dx + dy * dy + dz * dz);
-        fc = cutoff_f(d, rp.r_c);
+        if (d < rp.r_c) fc = 0.5f * (__cosf(pi_rc * d) + 1.f);  // argument in [0, pi)
       }
       M->src[t] = j;
       M->fc[t] = fc;
@@ -221,11 +222,16 @@ __global__ void __launch_bounds__(AT_THREADS, 1) k_attn_tc(
         M->first = (it % TPA) == 0;
         M->last = (it % TPA) == TPA - 1;
       }
-      // Gaussian operand row (bf16), bias column R = 1; zero for a padded slot
-      const float d0 = d - rp.mu_min;
+      // Gaussian operand row (bf16), bias column R = 1; zero for a padded slot. e_k = 2^(-x_k^2)
+      // on the scaled distance, by the two-ex2-per-eight-centres recurrence of the cfconv
+      // forward (tc_cfconv_ws.cu)
+      const float xk00 = (d - rp.mu_min) * xs;
       uint8_t* A = AB(b);
 #pragma unroll
       for (int k0 = 0; k0 < K1; k0 += 8) {
+        const float xk0 = fmaf(-(float)k0, dmu_x, xk00);
+        float ek = tc::ex2f(-(xk0 * xk0));
+        float rk = tc::ex2f(dmu_x * fmaf(2.f, xk0, -dmu_x));
         uint32_t w[4];
 #pragma unroll
         for (int qq = 0; qq < 4; ++qq) {
@@ -233,10 +239,11 @@ __global__ void __launch_bounds__(AT_THREADS, 1) k_attn_tc(
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             const int k = k0 + 2 * qq + hh;
-            const float dd = fmaf(-(float)k, rp.dmu, d0);
-            float val = tc::ex2f(nglog2e * dd * dd);
+            float val = ek;
             if (k >= K1 - 16) val = k < rp.R ? val : (k == rp.R ? 1.f : 0.f);
             v[hh] = ok ? val : 0.f;
+            ek *= rk;
+            rk *= rstep;
           }
           w[qq] = tc::pack_bf16(v[0], v[1]);
         }

@@ -176,7 +176,8 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_cfconv_fwd_ws(
   if (warp < PREP_WARPS) {
     // =============================================================== prep role (128 threads)
     const int t = tid;
-    const float nglog2e = -rp.gamma * LOG2E;
+    const float xs = sqrtf(rp.gamma * LOG2E), dmu_x = rp.dmu * xs;
+    const float rstep = tc::ex2f(-2.f * dmu_x * dmu_x), pi_rc = 3.14159265358979f / rp.r_c;
     int r_lo = r_begin;
     // the x_j rows of tile k, once every epilogue warp has read those of tile k-1 (16 threads per
     // 256-byte row); false on abort, uniformly over the prep warps
@@ -252,7 +253,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_cfconv_fwd_ws(
         if (jok) {
           const float dx = pix - pjx, dy = piy - pjy, dz = piz - pjz;
           d = sqrtf(dx * dx + dy * dy + dz * dz);
-          fc = cutoff_f(d, rp.r_c);
+          if (d < rp.r_c) fc = 0.5f * (__cosf(pi_rc * d) + 1.f);  // argument in [0, pi)
           ok = true;
         } else {
           raise_status(status, kStatusBounds);
@@ -261,11 +262,18 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_cfconv_fwd_ws(
       M->src[t] = j;
       M->fc[t] = fc;
       s_pdst[t] = my_dst;
-      // Gaussian operand row (bf16), bias column R = 1, zero padding
-      const float d0 = d - rp.mu_min;
+      // Gaussian operand row (bf16), bias column R = 1, zero padding. On the scaled distance
+      // x_k = (d - mu_k) sqrt(gamma log2 e), e_k = 2^(-x_k^2); within a chunk of eight centres
+      // e_{k+1} = e_k r_k, r_k = 2^(2 x_k dx - dx^2), r_{k+1} = r_k 2^(-2 dx^2): two ex2 per chunk
+      // (the relative error grows by a few ulp per step, far below the operand's bf16 rounding;
+      // where e_k0 underflows to 0 the chunk is below 2^-70, and r stays finite for |x| <= 80)
+      const float xk00 = (d - rp.mu_min) * xs;
       uint8_t* A = AB(it % NA);
 #pragma unroll
       for (int k0 = 0; k0 < K1; k0 += 8) {
+        const float xk0 = fmaf(-(float)k0, dmu_x, xk00);
+        float ek = tc::ex2f(-(xk0 * xk0));
+        float rk = tc::ex2f(dmu_x * fmaf(2.f, xk0, -dmu_x));
         uint32_t w[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -273,10 +281,11 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_cfconv_fwd_ws(
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             const int k = k0 + 2 * q + hh;
-            const float dd = fmaf(-(float)k, rp.dmu, d0);
-            float val = tc::ex2f(nglog2e * dd * dd);
+            float val = ek;
             if (k >= K1 - 16) val = k < rp.R ? val : (k == rp.R ? 1.f : 0.f);
             v[hh] = ok ? val : 0.f;
+            ek *= rk;
+            rk *= rstep;
           }
           w[q] = tc::pack_bf16(v[0], v[1]);
         }
