@@ -159,8 +159,7 @@ extern "C" int mp_attn_eq_fwd(mp_ctx* c, int N, int K, const float* pos, const i
   cudaStream_t s = (cudaStream_t)stream;
   const int F = c->cfg.F;
   const bool bf = c->cfg.dtype == MP_BF16;
-  int rc = launch_dense(c, N, F, F, x, bf, c->Wq, nullptr, false, c->q, false, s);
-  if (rc == MP_OK) rc = launch_dense(c, N, F, F, x, bf, c->Wk, nullptr, false, c->k, false, s);
+  int rc = attn_project(c, N, x, s);
   if (rc != MP_OK) return rc;
   if (tc_attn_eq_supported(c, K)) return tc_attn_eq_fwd(c, N, K, pos, nbr, mask, x, out, s);
   if (F == 64)

@@ -59,6 +59,7 @@ struct mp_ctx {
   void* tc_weights = nullptr;
   size_t tc_weights_bytes = 0;
   uint8_t* tc_dense_img = nullptr;        // packed bf16 atomwise weights (tc_dense.cu)
+  bool tc_qk = false;                     // tc_dense_img also holds the attention's Wq, Wk
   uint8_t* tc_attn_p = nullptr;           // attention: [16 heads][K1] bf16 P^T with p on column R
   // workspace, sized from max_atoms
   float* x_res = nullptr;                 // [N][F] fp32 residual stream

@@ -68,9 +68,14 @@ int tc_dense2(mp_ctx* ctx, int N, int K1, const void* in1, bool in1_bf16, const 
               void* out2, int mode2, cudaStream_t s);
 // Offsets of the packed dense images inside ctx->tc_dense_img.
 inline size_t tc_dense_off(int kind, int block, int n_blocks) {
-  // kind: 0 W_in, 1 W_out, 2 W_out^T, 3 W_in^T (per block), 4 B1, 5 B1^T
+  // kind: 0 W_in, 1 W_out, 2 W_out^T, 3 W_in^T (per block), 4 B1, 5 B1^T, 6 Wq, 7 Wk
   const size_t sq = (size_t)128 * 128 * 2;
   if (kind < 4) return ((size_t)block * 4 + kind) * sq;
+  if (kind >= 6) return ((size_t)n_blocks * 4 + 1 + (kind - 6)) * sq;
   return (size_t)n_blocks * 4 * sq + (kind == 4 ? 0 : sq / 2);
 }
+// The attention's query and key rows q = x Wq, k = x Wk (fp32 [N][F] in ctx->q, ctx->k): on the
+// tensor cores when the context holds their packed images (bf16 path, F = 128), else on the CUDA
+// cores (tc_dense.cu).
+int attn_project(mp_ctx* ctx, int N, const void* x, cudaStream_t s);
 }  // namespace mp

@@ -450,6 +450,14 @@ int tc_prepare(mp_ctx* ctx, cudaStream_t s) {
       return MP_ERR_CUDA;
     tc_dense_pack(B1.data(), FT, FT / 2, false, dimg.data() + tc_dense_off(4, 0, B));
     tc_dense_pack(B1.data(), FT, FT / 2, true, dimg.data() + tc_dense_off(5, 0, B));
+    if (c.n_heads > 0 && ctx->Wq && ctx->Wk) {  // the attention's query and key projections
+      if (cudaMemcpy(Wi.data(), ctx->Wq, Wi.size() * 4, cudaMemcpyDeviceToHost) != cudaSuccess ||
+          cudaMemcpy(Wo.data(), ctx->Wk, Wo.size() * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return MP_ERR_CUDA;
+      tc_dense_pack(Wi.data(), FT, FT, false, dimg.data() + tc_dense_off(6, 0, B));
+      tc_dense_pack(Wo.data(), FT, FT, false, dimg.data() + tc_dense_off(7, 0, B));
+      ctx->tc_qk = true;
+    }
     if (cudaMalloc(&ctx->tc_dense_img, dimg.size()) != cudaSuccess) return MP_ERR_CUDA;
     if (cudaMemcpy(ctx->tc_dense_img, dimg.data(), dimg.size(), cudaMemcpyHostToDevice) != cudaSuccess)
       return MP_ERR_CUDA;

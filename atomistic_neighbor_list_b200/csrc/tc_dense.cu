@@ -392,8 +392,8 @@ __global__ void __launch_bounds__(D2THREADS) k_dense2_tc(Dense2Args a, int* stat
 }  // namespace
 
 // Packed dense weight images in ctx->tc_dense: per block W_in, W_out, W_out^T, W_in^T (each
-// [128][128]), then B1 ([64][128]) and B1^T ([128][64]).
-size_t tc_dense_bytes(int B) { return (size_t)(4 * B + 1) * 128 * 128 * 2; }
+// [128][128]), then B1 ([64][128]) and B1^T ([128][64]), then the attention's Wq and Wk.
+size_t tc_dense_bytes(int B) { return (size_t)(4 * B + 3) * 128 * 128 * 2; }
 
 int tc_dense_pack(const float* W, int rows, int cols, bool transpose, uint8_t* dst) {
   // B operand [Nout][Kin]: element (n, k) = transpose ? W[n][k] : W[k][n], W row-major [rows][cols]
@@ -407,6 +407,21 @@ int tc_dense_pack(const float* W, int rows, int cols, bool transpose, uint8_t* d
       memcpy(dst + kmaj(n, k, Kin), &bits, 2);
     }
   return MP_OK;
+}
+
+int attn_project(mp_ctx* ctx, int N, const void* x, cudaStream_t s) {
+  const int F = ctx->cfg.F, B = ctx->cfg.n_blocks;
+  const bool bf = ctx->cfg.dtype == MP_BF16;
+  if (ctx->tc_qk && ((uintptr_t)x & 15) == 0) {  // bf16 rows x bf16 weights, fp32 accumulation
+    int rc = tc_dense(ctx, N, F, F, x, true, ctx->tc_dense_img + tc_dense_off(6, 0, B), nullptr,
+                      ctx->q, false, TC_DENSE_STORE, s);
+    if (rc != MP_OK) return rc;
+    return tc_dense(ctx, N, F, F, x, true, ctx->tc_dense_img + tc_dense_off(7, 0, B), nullptr,
+                    ctx->k, false, TC_DENSE_STORE, s);
+  }
+  int rc = launch_dense(ctx, N, F, F, x, bf, ctx->Wq, nullptr, false, ctx->q, false, s);
+  if (rc != MP_OK) return rc;
+  return launch_dense(ctx, N, F, F, x, bf, ctx->Wk, nullptr, false, ctx->k, false, s);
 }
 
 int tc_dense(mp_ctx* ctx, int N, int Kin, int Nout, const void* in, bool in_bf16, const uint8_t* wimg,
