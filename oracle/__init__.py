@@ -32,7 +32,7 @@ only by the written specification that both this oracle and the CUDA path follow
 from .neighbors import cutoff_sq, pair_d2, neighbor_csr, neighbor_padded  # noqa: F401
 from .schnet import (  # noqa: F401
     LN2, rbf_centres, gaussian_rbf, gaussian_rbf_grad, cosine_cutoff, cosine_cutoff_grad, ssp,
-    ssp_grad, filter_weights, cfconv, Model, energies, energy_forces,
+    ssp_grad, filter_weights, cfconv, cfconv_pairs, undirected_pairs, Model, energies, energy_forces,
 )
 from .attention import (  # noqa: F401
     attention, attention_vjp, attention_equivariant, solid_harmonics, moments_to_solid,

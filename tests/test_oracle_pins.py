@@ -231,6 +231,75 @@ def test_cfconv_reduces_to_dense_spmm():
     assert np.allclose(m, A @ x.astype(float), rtol=1e-12, atol=1e-12)
 
 
+def test_pair_cfconv_two_atoms_by_hand():
+    # one pair: the filter once, x_1 (.) W to row 0 and x_0 (.) W to row 1 (the hand formula above)
+    model, w, wl = small_model(F=4, R=5)
+    pos = np.array([[0.1, 0.2, 0.3], [1.0, 2.0, 2.5]], dtype=np.float32)
+    x = synth.node_features(2, 4, seed=9)
+    rp, ci = oracle.neighbor_csr(pos, 5.0)
+    m = oracle.cfconv_pairs(model, 0, pos, rp, ci, x)
+    p = pos.astype(float)
+    d = math.sqrt(sum((p[0, c] - p[1, c]) ** 2 for c in range(3)))
+    e = [math.exp(-10.0 * (d - 5.0 * k / 4) ** 2) for k in range(5)]
+    A1, c1, A2, c2 = (w[k].astype(float) for k in ("A1.0", "c1.0", "A2.0", "c2.0"))
+    h1 = [math.log(0.5 * math.exp(sum(e[k] * A1[k, g] for k in range(5)) + c1[g]) + 0.5)
+          for g in range(4)]
+    fc = 0.5 * (math.cos(math.pi * d / 5.0) + 1.0)
+    W = [fc * (sum(h1[g] * A2[g, f] for g in range(4)) + c2[f]) for f in range(4)]
+    assert np.allclose(m[0], [x[1, f] * W[f] for f in range(4)], rtol=1e-12, atol=1e-14)
+    assert np.allclose(m[1], [x[0, f] * W[f] for f in range(4)], rtol=1e-12, atol=1e-14)
+
+
+def test_pair_cfconv_reduces_to_symmetric_spmm():
+    # W = f_c  =>  m = A x with A symmetric, A_ij = f_c(d_ij) on neighbor pairs
+    model, w, wl = small_model(F=8)
+    model.w["A1.0"][:] = 0
+    model.w["A2.0"][:] = 0
+    model.w["c2.0"][:] = 1
+    pos = synth.uniform_positions(150, seed=2)
+    x = synth.node_features(150, 8, seed=1)
+    rp, ci = brute_csr(pos, 5.0)
+    A = np.zeros((150, 150))
+    p = pos.astype(float)
+    for i in range(150):
+        for j in ci[rp[i]:rp[i + 1]]:
+            d = math.sqrt(sum((p[i, c] - p[j, c]) ** 2 for c in range(3)))
+            A[i, j] = 0.5 * (math.cos(math.pi * d / 5.0) + 1.0)
+    assert np.array_equal(A, A.T)
+    m = oracle.cfconv_pairs(model, 0, pos, rp, ci, x)
+    assert np.allclose(m, A @ x.astype(float), rtol=1e-12, atol=1e-12)
+
+
+def test_pair_cfconv_evaluates_each_filter_once(monkeypatch):
+    # the pair form calls the filter on E / 2 distances and gives the directed form's sums
+    model, w, wl = small_model(F=8)
+    pos = synth.uniform_positions(300, seed=6)
+    x = synth.node_features(300, 8, seed=3)
+    rp, ci = oracle.neighbor_csr(pos, 5.0)
+    seen = []
+    real = oracle.schnet.filter_weights
+
+    def counting(model_, b, d, with_grad=False):
+        seen.append(len(d))
+        return real(model_, b, d, with_grad)
+
+    monkeypatch.setattr(oracle.schnet, "filter_weights", counting)
+    m_pair = oracle.cfconv_pairs(model, 0, pos, rp, ci, x)
+    assert sum(seen) * 2 == len(ci) and len(ci) > 1000
+    monkeypatch.setattr(oracle.schnet, "filter_weights", real)
+    m_dir = oracle.cfconv(model, 0, pos, rp, ci, x)
+    assert np.allclose(m_pair, m_dir, rtol=1e-12, atol=1e-12)
+
+
+def test_undirected_pairs_need_a_symmetric_list():
+    rp = np.array([0, 1, 1, 2])
+    ci = np.array([1, 0])  # 1 -> 0 and 0 -> 2: the reverse of 0 -> 2 is missing
+    with pytest.raises(ValueError):
+        oracle.undirected_pairs(rp, ci)
+    i, j = oracle.undirected_pairs(np.array([0, 2, 3, 4]), np.array([1, 2, 0, 0]))
+    assert i.tolist() == [0, 0] and j.tolist() == [1, 2]
+
+
 def test_cfconv_empty_rows_and_permutation():
     model, w, wl = small_model(F=8)
     pos = synth.uniform_positions(120, seed=5)
