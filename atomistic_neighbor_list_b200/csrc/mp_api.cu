@@ -17,7 +17,7 @@ const char* kernel_name(int id) {
       "attn_tc", "dense_tc", "md_integrate", "attn_bwd_dst", "attn_bwd_src",
       "attn_transpose", "attn_eq_simt", "attn_bwd_dst_tc",
       "attn_bwd_src_tc", "attn_eq_tc", "md_cutoff_list", "cfconv_fwd_tc_lockstep",
-      "cfconv_bwd_tc_lockstep"};
+      "cfconv_bwd_tc_lockstep", "pair_plan", "cfconv_pair_tc", "pair_sum"};
   return (id >= 0 && id < K_NUM) ? names[id] : "?";
 }
 
@@ -95,6 +95,7 @@ void free_ctx(mp_ctx* c) {
   cudaFree(c->tc_dense_img);
   cudaFree(c->tc_attn_p);
   if (c->ef_graph) cudaGraphExecDestroy(c->ef_graph);
+  pair_plan_free(c);
   cudaFree(c->x_res);  // one allocation holds the whole workspace
   cudaFree(c->status_d);
   if (c->status_h) cudaFreeHost(c->status_h);
@@ -312,6 +313,30 @@ extern "C" int mp_cfconv_fwd(mp_ctx* c, int block, int N, long long E, const flo
   if (N == 0) return MP_OK;
   if (tc_supported(c)) return tc_cfconv_fwd(c, block, N, E, pos, row_ptr, col_idx, x, out, s);
   return launch_cfconv_fwd_simt(c, block, N, E, pos, row_ptr, col_idx, x, out, s);
+}
+
+extern "C" int mp_pair_plan(mp_ctx* c, int N, long long E, const int* row_ptr,
+                            const int* col_idx, void* stream) {
+  if (!c || N < 0 || E < 0 || !row_ptr || (E > 0 && !col_idx)) return MP_ERR_INVALID_ARG;
+  if (N > c->cfg.max_atoms || E > c->cfg.max_edges) return MP_ERR_CAPACITY;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (c->cfg.validate) {
+    int rc = launch_validate_csr(c, N, E, row_ptr, col_idx, nullptr, 1, true, s);
+    if (rc != MP_OK) return rc;
+  }
+  return pair_plan_build(c, N, E, row_ptr, col_idx, s);
+}
+
+extern "C" int mp_cfconv_fwd_pairs(mp_ctx* c, int block, int N, const float* pos, const void* x,
+                                   void* out, void* stream) {
+  if (!c || block < 0 || block >= c->cfg.n_blocks || N < 0 ||
+      (N > 0 && (!pos || !x || !out)) || (x && x == out) || ((uintptr_t)x & 15) != 0 ||
+      ((uintptr_t)out & 15) != 0)
+    return MP_ERR_INVALID_ARG;
+  if (!tc_supported(c)) return MP_ERR_UNIMPLEMENTED;
+  if (!c->pair.valid || c->pair.N != N) return MP_ERR_INVALID_ARG;
+  if (N == 0) return MP_OK;
+  return tc_cfconv_fwd_pairs(c, block, N, pos, x, out, (cudaStream_t)stream);
 }
 
 extern "C" int mp_attn_fwd(mp_ctx* c, int N, int K, const float* pos, const int* nbr,

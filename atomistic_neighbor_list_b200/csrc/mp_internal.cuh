@@ -36,9 +36,45 @@ enum KernelId : int {
   K_CFCONV_BWD_SIMT, K_ATTN_SIMT, K_VALIDATE, K_CFCONV_FWD_TC, K_CFCONV_BWD_TC, K_ATTN_TC,
   K_DENSE_TC, K_MD, K_ATTN_BWD, K_ATTN_BWD_SRC, K_ATTN_REV, K_ATTN_EQ,
   K_ATTN_BWD_TC, K_ATTN_BWD_SRC_TC, K_ATTN_EQ_TC, K_MD_CUT, K_CFCONV_FWD_TC_LS,
-  K_CFCONV_BWD_TC_LS, K_NUM
+  K_CFCONV_BWD_TC_LS, K_PAIR_PLAN, K_CFCONV_PAIR_TC, K_PAIR_SUM, K_NUM
 };
 const char* kernel_name(int id);
+
+// One tile of the undirected-pair cfconv (pairs.cu, tc_cfconv_pair.cu): 128 pair slots of the
+// block pair (I, J) of 128-atom blocks, and how the kernel's accumulators m_I, m_J treat it.
+enum : int {
+  kPairAccI = 1,     // add to m_I (0: this tile starts a run of m_I)
+  kPairAccJ = 2,     // add to m_J (0: this tile starts a run of m_J)
+  kPairDiag = 4,     // I == J: both messages go to m_I
+  kPairFlushI = 8,   // the run of m_I ends here: written to partial slotI
+  kPairFlushJ = 16   // the run of m_J ends here: written to partial slotJ
+};
+struct PairTile {
+  int I, J, count, flags, slotI, slotJ, pad0, pad1;
+};
+constexpr int kPairF = 128;  // features of the pair path (the tensor-core configuration)
+
+// The plan of one symmetric neighbor list (pairs.cu); device arrays in one allocation.
+struct PairPlan {
+  bool valid = false;
+  int N = 0, NB = 0, G = 0, T = 0, nslots = 0;
+  long long E = 0;
+  void* ws = nullptr;      // per-block arrays (sized by E and the number of blocks)
+  size_t ws_bytes = 0;
+  void* tws = nullptr;     // the tiles (sized by their count)
+  size_t tws_bytes = 0;
+  float* part = nullptr;  // [nslots][128 rows][128 features] fp32 partial rows
+  uint32_t* pmask = nullptr;  // [nslots][4]: the rows each partial block holds (the rest unset)
+  size_t part_bytes = 0;
+  int2* pairs = nullptr;  // per block, at pbase[R]: its upper pairs sorted by (J, i, j)
+  int4* segs = nullptr;   // per block, at pbase[R]: (J, first pair, pairs, first local tile)
+  int* low = nullptr;     // per block, at pbase[R]: the blocks J < R that hold neighbors
+  int *pbase = nullptr, *nseg = nullptr, *ntile = nullptr, *nlow = nullptr, *toff = nullptr;
+  int2* tpairs = nullptr; // [T][128] pair slots (i, j), (-1, -1) on padding
+  PairTile* tiles = nullptr;
+  int *sum_cnt = nullptr, *sum_ptr = nullptr, *sum_slots = nullptr;  // summing lists per block
+  int* counts = nullptr;
+};
 
 }  // namespace mp
 
@@ -94,6 +130,8 @@ struct mp_ctx {
     const void *pos, *types, *row_ptr, *col_idx, *graph_ptr;
     void *energy, *forces, *stream;
   } ef_key{};
+  // undirected-pair plan of the last list given to mp_pair_plan
+  mp::PairPlan pair;
   // profiling
   bool profiling = false;
   std::vector<cudaEvent_t> ev_pool;
@@ -220,6 +258,16 @@ void launch_scan(long long n, int* a, long long* bsum, int* overflow, cudaStream
 int energy_forces_launches(mp_ctx*, int N, long long E, const float* pos, const int* types,
                            const int* row_ptr, const int* col_idx, const int* graph_ptr,
                            int n_graphs, float* energy, float* forces, cudaStream_t);
+
+// Undirected-pair cfconv (pairs.cu, tc_cfconv_pair.cu): build the plan of a symmetric list
+// (synchronises the stream), the pair kernel, and the fixed-order sum of its partial rows.
+int pair_plan_build(mp_ctx*, int N, long long E, const int* row_ptr, const int* col_idx,
+                    cudaStream_t);
+int pair_sum_launch(mp_ctx*, int N, void* out, cudaStream_t);
+int tc_cfconv_fwd_pairs(mp_ctx*, int block, int N, const float* pos, const void* x, void* out,
+                        cudaStream_t);
+void pair_plan_free(mp_ctx*);
+inline size_t align_up_sz(size_t v) { return (v + 255) / 256 * 256; }
 
 FilterW filter_of(const mp_ctx* ctx, int block);
 Radial radial_of(const mp_ctx* ctx);

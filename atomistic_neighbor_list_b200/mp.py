@@ -66,6 +66,8 @@ def _load():
         "mp_profile_get": (i32, [vp, i32, POINTER(c_char_p), POINTER(c_double), POINTER(i64)]),
         "mp_launch_count": (i64, [vp]),
         "mp_set_wait_budget": (i32, [vp, i64]),
+        "mp_pair_plan": (i32, [vp, i32, i64, vp, vp, vp]),
+        "mp_cfconv_fwd_pairs": (i32, [vp, i32, i32, vp, vp, vp, vp]),
         "mp_set_graphs": (i32, [vp, i32]),
         "mp_md_verlet": (i32, [vp, i32, i64, vp, vp, vp, vp, c_float, i32, vp, vp, vp, vp, i32,
                                vp, vp, vp]),
@@ -92,7 +94,7 @@ EXPORTED = ("mp_init", "mp_destroy", "mp_strerror", "mp_status_sync", "mp_neighb
             "mp_profile_begin", "mp_profile_end", "mp_profile_get", "mp_launch_count",
             "mp_attn_fwd_noalloc", "mp_selftest_tc", "mp_set_graphs",
             "mp_md_verlet", "mp_md_run", "mp_attn_bwd", "mp_attn_eq_fwd", "mp_spatial_order",
-            "mp_set_wait_budget")
+            "mp_set_wait_budget", "mp_pair_plan", "mp_cfconv_fwd_pairs")
 NOALLOC_MAX_NF = 524288  # MP_NOALLOC_MAX_NF: largest N * F mp_attn_fwd_noalloc accepts
 
 
@@ -200,6 +202,26 @@ class Context:
         _check(lib.mp_cfconv_fwd(self._ctx, block, N, col_idx.numel(), _ptr(pos), _ptr(row_ptr),
                                  _ptr(col_idx), _ptr(x), _ptr(out), _stream(stream)),
                "mp_cfconv_fwd")
+        return out
+
+    def pair_plan(self, row_ptr, col_idx, stream=None):
+        """Undirected-pair plan of a symmetric CSR for cfconv_fwd_pairs (synchronises)."""
+        N = row_ptr.numel() - 1
+        _need(row_ptr, "row_ptr", torch.int32, (N + 1,))
+        _need(col_idx, "col_idx", torch.int32)
+        _check(lib.mp_pair_plan(self._ctx, N, col_idx.numel(), _ptr(row_ptr), _ptr(col_idx),
+                                _stream(stream)), "mp_pair_plan")
+
+    def cfconv_fwd_pairs(self, block, pos, x, out=None, stream=None):
+        """cfconv_fwd over the pairs of the last pair_plan: one filter per undirected pair."""
+        N = x.shape[0]
+        _need(pos, "pos", torch.float32, (N, 3))
+        _need(x, "x", self.tdtype, (N, self.F))
+        if out is None:
+            out = torch.empty_like(x)
+        _need(out, "out", self.tdtype, (N, self.F))
+        _check(lib.mp_cfconv_fwd_pairs(self._ctx, block, N, _ptr(pos), _ptr(x), _ptr(out),
+                                       _stream(stream)), "mp_cfconv_fwd_pairs")
         return out
 
     def attn_fwd(self, pos, nbr, mask, x, out=None, stream=None):

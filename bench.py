@@ -422,6 +422,16 @@ def measure_configs(keys, devn, stream, flush, steps: int):
         ms_blk = timed(blk, n_calls)
         res = {"workload": wl.name, "atoms": N, "edges": E, "dtype": wl.dtype,
                "block_edges_per_s": E / (ms_blk / 1000.0), "ms_per_block": ms_blk}
+        if wl.dtype == "bf16" and wl.F == 128:  # the filter once per undirected pair
+            t0 = time.perf_counter()
+            ctx.pair_plan(rp, ci)
+            plan_ms = (time.perf_counter() - t0) * 1000.0
+            pblk = lambda: ctx.cfconv_fwd_pairs(0, pos_d, x, m)
+            for _ in range(3):
+                pblk()
+            ms_p = timed(pblk, n_calls)
+            res["pair_filter"] = {"block_edges_per_s": E / (ms_p / 1000.0), "ms_per_block": ms_p,
+                                  "plan_ms": plan_ms}
         if wl.kind == "cfconv":
             profs[key] = (profiled(ctx, blk, 5), wl, E, N, ms_blk)
         else:
@@ -596,6 +606,28 @@ def main():
     torch.cuda.synchronize()
     cf_total = sum(a.elapsed_time(b) for a, b in cf_ms) / len(cf_ms)
     edges_per_s = E / (cf_total / 1000.0)
+    # the same block with the filter evaluated once per undirected pair (plan built once)
+    pair_blk = None
+    if wl.dtype == "bf16" and wl.F == 128 and not args.profile_run:
+        t0 = time.perf_counter()
+        ctx.pair_plan(rp, ci)
+        plan_ms = (time.perf_counter() - t0) * 1000.0
+        for _ in range(3):
+            ctx.cfconv_fwd_pairs(0, pos_d, x_in, out_m)
+        pe = []
+        for _ in range(max(10, args.steps)):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            ctx.cfconv_fwd_pairs(0, pos_d, x_in, out_m)
+            b.record(stream)
+            pe.append((a, b))
+        torch.cuda.synchronize()
+        ms_p = sum(a.elapsed_time(b) for a, b in pe) / len(pe)
+        pair_blk = {"value": E / (ms_p / 1000.0), "unit": "edges/s", "ms_per_block": ms_p,
+                    "plan_ms": plan_ms, "call": "mp_cfconv_fwd_pairs: filter once per "
+                    "undirected pair, then the fixed-order sum of the partial rows; plan by "
+                    "mp_pair_plan, once per neighbor list (wall clock, two host syncs)"}
 
     # ---- attention variant (cfg4: 32,768 atoms, padded K = 256): edges/s counting valid edges,
     # same timing rules; q and k projections included
@@ -828,7 +860,8 @@ def main():
                "md_loop": md,
                "edges_per_s_per_block": {"value": edges_per_s, "unit": "edges/s",
                                          "ms_per_block": cf_total,
-                                         "cpu_baseline": cpu_extra.get("cfg2_block")},
+                                         "cpu_baseline": cpu_extra.get("cfg2_block"),
+                                         "pair_filter": pair_blk},
                "cpu_legs": cpu_extra.get("cfg2_energy_forces"),
                "configs": configs,
                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,

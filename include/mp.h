@@ -169,6 +169,31 @@ int mp_spatial_order(int N, const float* pos, const int* graph_ptr, int n_graphs
 int mp_cfconv_fwd(mp_ctx* ctx, int block, int N, long long E, const float* pos,
                   const int* row_ptr, const int* col_idx, const void* x, void* out, void* stream);
 
+/* Undirected-pair plan of a symmetric neighbor list [FS s.2.3: the symmetric list; s.2.4: the
+ * filter MLP], kept in the context for mp_cfconv_fwd_pairs: the pairs {i, j} (i < j) once each,
+ * grouped by blocks of 128 atoms into tiles of 128 pairs of one block pair, and the order in
+ * which the pair kernel's partial rows are summed. Built on the device from the CSR (which must
+ * be symmetric, as any cutoff list is: with validate set this is checked first); the plan does
+ * not hold the positions, so it stays valid for every configuration the same list serves.
+ * Workspace: O(E) ints plus one 64 KiB fp32 partial block per run of tiles, allocated here
+ * (grown when a larger list comes) and freed by mp_destroy. Synchronises `stream`.
+ * Errors: MP_ERR_INVALID_ARG, MP_ERR_CAPACITY (more than 32768 upper pairs of one 128-atom
+ * block, more than 1024 block pairs of one block, or N > 8388608), MP_ERR_DEVICE_BOUNDS (a
+ * column index outside [0, N)), MP_ERR_CUDA, CSR errors (validate).                            */
+int mp_pair_plan(mp_ctx* ctx, int N, long long E, const int* row_ptr, const int* col_idx,
+                 void* stream);
+
+/* mp_cfconv_fwd over the pairs of the current plan: the filter W(d_ij) = W(d_ji) evaluated once
+ * per pair and both messages taken from it, x_j (.) W to row i and x_i (.) W to row j, on the
+ * tensor cores; each row written once by a fixed-order sum of per-run fp32 partials (no
+ * atomics, results bitwise repeatable). Same out as mp_cfconv_fwd on the plan's list. Needs the
+ * bf16 tensor-core configuration (F = 128) and a plan of the same N (the list of the last
+ * mp_pair_plan call). x, out: [N][F] bf16, 16-byte aligned, out must not alias x.
+ * Errors: MP_ERR_INVALID_ARG (no plan, another N, misaligned x or out), MP_ERR_UNIMPLEMENTED
+ * (fp32 or another F), MP_ERR_CUDA.                                                           */
+int mp_cfconv_fwd_pairs(mp_ctx* ctx, int block, int N, const float* pos, const void* x,
+                        void* out, void* stream);
+
 /* Neighbor attention aggregation with an online softmax [E2 s.3.1-3.2]. With q = x Wq,
  * k = x Wk split into n_heads heads of head_dim channels, for each valid slot j of row i
  * (mask != 0 and 0 <= nbr < N):
