@@ -159,9 +159,10 @@ extern "C" int mp_attn_eq_fwd(mp_ctx* c, int N, int K, const float* pos, const i
   cudaStream_t s = (cudaStream_t)stream;
   const int F = c->cfg.F;
   const bool bf = c->cfg.dtype == MP_BF16;
-  int rc = attn_project(c, N, x, s);
+  const bool tc = tc_attn_eq_supported(c, K) && ((uintptr_t)x & 15) == 0;
+  int rc = attn_project(c, N, x, s, tc);
   if (rc != MP_OK) return rc;
-  if (tc_attn_eq_supported(c, K)) return tc_attn_eq_fwd(c, N, K, pos, nbr, mask, x, out, s);
+  if (tc) return tc_attn_eq_fwd(c, N, K, pos, nbr, mask, x, out, s);
   if (F == 64)
     return bf ? run_attn_eq<__nv_bfloat16, 64>(c, N, K, pos, nbr, mask, x, out, s)
               : run_attn_eq<float, 64>(c, N, K, pos, nbr, mask, x, out, s);

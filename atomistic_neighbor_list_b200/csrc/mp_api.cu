@@ -347,9 +347,10 @@ extern "C" int mp_attn_fwd(mp_ctx* c, int N, int K, const float* pos, const int*
   if (N > c->cfg.max_atoms) return MP_ERR_CAPACITY;
   if (N == 0) return MP_OK;
   cudaStream_t s = (cudaStream_t)stream;
-  int rc = attn_project(c, N, x, s);
+  const bool tc = tc_attn_supported(c, K) && ((uintptr_t)x & 15) == 0;
+  int rc = attn_project(c, N, x, s, tc);
   if (rc != MP_OK) return rc;
-  if (tc_attn_supported(c, K)) return tc_attn_fwd(c, N, K, pos, nbr, mask, x, out, s);
+  if (tc) return tc_attn_fwd(c, N, K, pos, nbr, mask, x, out, s);
   return launch_attn_simt(c, N, K, pos, nbr, mask, x, out, s);
 }
 

@@ -32,8 +32,9 @@ int tc_cfconv_bwd_ws(mp_ctx* ctx, int block, int N, long long E, const float* po
 int tc_cfconv_bwd(mp_ctx* ctx, int block, int N, long long E, const float* pos, const int* row_ptr,
                   const int* col_idx, const void* h, const void* g, float* grad_h, float* forces,
                   bool accumulate, cudaStream_t s);
-// Neighbor attention on the tensor cores (tc_attn.cu): 16 heads of 8, K a multiple of 128; q and
-// k (fp32 [N][F]) must already be in ctx->q, ctx->k.
+// Neighbor attention on the tensor cores (tc_attn.cu): 16 heads of 8, K a multiple of 128, x
+// 16-byte aligned; q (fp32 [N][F]) and k (fp16 [N][F], attn_project with k_f16) must already be in
+// ctx->q, ctx->k.
 bool tc_attn_supported(const mp_ctx* ctx, int K);
 int tc_attn_fwd(mp_ctx* ctx, int N, int K, const float* pos, const int* nbr,
                 const unsigned char* mask, const void* x, void* out, cudaStream_t s);
@@ -54,7 +55,7 @@ int tc_attn_bwd_src(mp_ctx* ctx, int N, int K, const float* pos, const int* rev_
                     const int* rev, const void* x, const float* g, float* grad_x, float* gk,
                     float* grad_pos, cudaStream_t s);
 // Atomwise layer on the tensor cores: out = in . W + b over rows (see tc_dense.cu for the modes).
-enum { TC_DENSE_STORE = 0, TC_DENSE_RESIDUAL = 1, TC_DENSE_READOUT = 2 };
+enum { TC_DENSE_STORE = 0, TC_DENSE_RESIDUAL = 1, TC_DENSE_READOUT = 2, TC_DENSE_STORE_F16 = 3 };
 size_t tc_dense_bytes(int n_blocks);
 int tc_dense_pack(const float* W, int rows, int cols, bool transpose, uint8_t* dst);
 int tc_dense(mp_ctx* ctx, int N, int Kin, int Nout, const void* in, bool in_bf16,
@@ -76,6 +77,7 @@ inline size_t tc_dense_off(int kind, int block, int n_blocks) {
 }
 // The attention's query and key rows q = x Wq, k = x Wk (fp32 [N][F] in ctx->q, ctx->k): on the
 // tensor cores when the context holds their packed images (bf16 path, F = 128), else on the CUDA
-// cores (tc_dense.cu).
-int attn_project(mp_ctx* ctx, int N, const void* x, cudaStream_t s);
+// cores (tc_dense.cu). k_f16: k stored as fp16 [N][F] instead (the tensor-core attention forward's
+// operand; needs the tensor-core projection).
+int attn_project(mp_ctx* ctx, int N, const void* x, cudaStream_t s, bool k_f16 = false);
 }  // namespace mp

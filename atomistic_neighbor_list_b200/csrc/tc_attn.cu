@@ -92,7 +92,7 @@ template <int K1, int NC>
 __global__ void __launch_bounds__(AT_THREADS, 1) k_attn_tc(
     int N, int K, const float* __restrict__ pos, const int* __restrict__ nbr,
     const unsigned char* __restrict__ mask, const __nv_bfloat16* __restrict__ x,
-    const float* __restrict__ q, const float* __restrict__ kx, __nv_bfloat16* __restrict__ out,
+    const float* __restrict__ q, const __half* __restrict__ kx, __nv_bfloat16* __restrict__ out,
     const uint8_t* __restrict__ img, const uint8_t* __restrict__ pimg, Radial rp, float qscale,
     int* status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -363,11 +363,11 @@ __global__ void __launch_bounds__(AT_THREADS, 1) k_attn_tc(
       AtRed* R = RB(b);
       const bool ok = M->ok[e_me] != 0;
       const float fc = M->fc[e_me];
-      // k_j of the 4 heads (fp32), requested before the waits
-      const float4* kr = (const float4*)(kx + (size_t)M->src[e_me] * FT + f0);
-      float4 kv[8];
+      // k_j of the 4 heads (fp16, 8 per 16-byte load), requested before the waits
+      const uint4* kr = (const uint4*)(kx + (size_t)M->src[e_me] * FT + f0);
+      uint4 kv[4];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) kv[c] = __ldg(kr + c);
+      for (int c = 0; c < 4; ++c) kv[c] = __ldg(kr + c);
       if (!wait_warp(B_XFULL, i & 1)) return false;
       uint4 xv[FPT / 8];
 #pragma unroll
@@ -380,15 +380,18 @@ __global__ void __launch_bounds__(AT_THREADS, 1) k_attn_tc(
       for (int hh = 0; hh < 4; ++hh) {
         const float4 qa = *(const float4*)(M->q + f0 + 8 * hh);
         const float4 qb = *(const float4*)(M->q + f0 + 8 * hh + 4);
-        const float4 ka = kv[2 * hh], kb = kv[2 * hh + 1];
-        float s = qa.x * ka.x;
-        s = fmaf(qa.y, ka.y, s);
-        s = fmaf(qa.z, ka.z, s);
-        s = fmaf(qa.w, ka.w, s);
-        s = fmaf(qb.x, kb.x, s);
-        s = fmaf(qb.y, kb.y, s);
-        s = fmaf(qb.z, kb.z, s);
-        s = fmaf(qb.w, kb.w, s);
+        const uint32_t kw[4] = {kv[hh].x, kv[hh].y, kv[hh].z, kv[hh].w};
+        float2 k2[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) k2[c] = __half22float2(*(const __half2*)&kw[c]);
+        float s = qa.x * k2[0].x;
+        s = fmaf(qa.y, k2[0].y, s);
+        s = fmaf(qa.z, k2[1].x, s);
+        s = fmaf(qa.w, k2[1].y, s);
+        s = fmaf(qb.x, k2[2].x, s);
+        s = fmaf(qb.y, k2[2].y, s);
+        s = fmaf(qb.z, k2[3].x, s);
+        s = fmaf(qb.w, k2[3].y, s);
         l[hh] = ok ? s + bias[hh] : -INFINITY;
       }
       // the tile's maximum per head: over the warp, then over the 4 warps of this feature quarter
@@ -543,7 +546,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1) k_attn_tc(
 
 bool tc_attn_supported(const mp_ctx* ctx, int K) {
   const mp_config& c = ctx->cfg;
-  return tc_supported(ctx) && ctx->tc_attn_p && c.n_heads == AH && c.head_dim == AD &&
+  return tc_supported(ctx) && ctx->tc_attn_p && ctx->tc_qk && c.n_heads == AH && c.head_dim == AD &&
          K % TM == 0 && at_fits(k1_of(c.n_rbf), 1);
 }
 
@@ -560,7 +563,7 @@ int tc_attn_launch(mp_ctx* ctx, int N, int K, const float* pos, const int* nbr,
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     return launch(ctx, NC == 1 ? K_ATTN_TC : K_ATTN_EQ_TC, kern, dim3(grid), dim3(AT_THREADS),
                   smem, s, N, K, pos, nbr, mask, (const __nv_bfloat16*)x, (const float*)ctx->q,
-                  (const float*)ctx->k, (__nv_bfloat16*)out, img, (const uint8_t*)ctx->tc_attn_p,
+                  (const __half*)ctx->k, (__nv_bfloat16*)out, img, (const uint8_t*)ctx->tc_attn_p,
                   radial_of(ctx), qscale, ctx->status_d);
   };
   if (K1 == 64) return go(k_attn_tc<64, NC>, 64);

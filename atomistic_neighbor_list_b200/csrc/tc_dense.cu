@@ -18,7 +18,7 @@ using namespace tcc;
 constexpr int DT = 128;  // rows per tile
 constexpr int DTHREADS = 128;
 
-enum { MODE_STORE = 0, MODE_RESIDUAL = 1, MODE_READOUT = 2 };
+enum { MODE_STORE = 0, MODE_RESIDUAL = 1, MODE_READOUT = 2, MODE_STORE_F16 = 3 };
 
 // Row r of a bf16 or fp32 [*][Kin] input, as bf16, into row `lane` of a K-major operand tile (all
 // loads of a half issued before use); zeros for rows past the end.
@@ -183,6 +183,16 @@ __global__ void __launch_bounds__(DTHREADS) k_dense_tc(DenseArgs a, int* status)
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(rr[i]) + (a.bias ? a.bias[col + i] : 0.f);
           if (a.mode == MODE_READOUT) {
             e_acc += readout_cols(v, col, a.B2, (float*)a.out + (size_t)r * a.Nout + col);
+          } else if (a.mode == MODE_STORE_F16) {  // fp16 rows (10-bit mantissa)
+            uint4* o = (uint4*)((__half*)a.out + (size_t)r * a.Nout + col);
+            auto h2 = [](float lo, float hi) {
+              const __half2 h = __floats2half2_rn(lo, hi);
+              return *(const uint32_t*)&h;
+            };
+#pragma unroll
+            for (int i = 0; i < 32; i += 8)
+              o[i / 8] = make_uint4(h2(v[i], v[i + 1]), h2(v[i + 2], v[i + 3]),
+                                    h2(v[i + 4], v[i + 5]), h2(v[i + 6], v[i + 7]));
           } else if (a.out_bf16) {
             uint4* o = (uint4*)((__nv_bfloat16*)a.out + (size_t)r * a.Nout + col);
 #pragma unroll
@@ -409,7 +419,7 @@ int tc_dense_pack(const float* W, int rows, int cols, bool transpose, uint8_t* d
   return MP_OK;
 }
 
-int attn_project(mp_ctx* ctx, int N, const void* x, cudaStream_t s) {
+int attn_project(mp_ctx* ctx, int N, const void* x, cudaStream_t s, bool k_f16) {
   const int F = ctx->cfg.F, B = ctx->cfg.n_blocks;
   const bool bf = ctx->cfg.dtype == MP_BF16;
   if (ctx->tc_qk && ((uintptr_t)x & 15) == 0) {  // bf16 rows x bf16 weights, fp32 accumulation
@@ -417,8 +427,9 @@ int attn_project(mp_ctx* ctx, int N, const void* x, cudaStream_t s) {
                       ctx->q, false, TC_DENSE_STORE, s);
     if (rc != MP_OK) return rc;
     return tc_dense(ctx, N, F, F, x, true, ctx->tc_dense_img + tc_dense_off(7, 0, B), nullptr,
-                    ctx->k, false, TC_DENSE_STORE, s);
+                    ctx->k, false, k_f16 ? TC_DENSE_STORE_F16 : TC_DENSE_STORE, s);
   }
+  if (k_f16) return MP_ERR_INVALID_ARG;  // the fp16 keys come from the tensor-core projection
   int rc = launch_dense(ctx, N, F, F, x, bf, ctx->Wq, nullptr, false, ctx->q, false, s);
   if (rc != MP_OK) return rc;
   return launch_dense(ctx, N, F, F, x, bf, ctx->Wk, nullptr, false, ctx->k, false, s);
