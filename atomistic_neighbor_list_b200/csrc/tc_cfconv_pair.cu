@@ -5,13 +5,14 @@
 //   MMA1   z1 = e . [A1; c1]                                   (the Gaussian operand of the pairs)
 //   E1     h' = f_c ssp(z1)
 //   MMA2   u = h' A2;  W = u + f_c c2 (one filter per pair)
-//   E2a    msg_I = x_j (.) W   ->  MMA3_I: m_I^T += msg_I^T S_I^T  (S_I: pair -> i mod 128)
-//   E2b    msg_J = x_i (.) W   ->  MMA3_J: m_J^T += msg_J^T S_J^T  (m_I when I = J)
+//   E2     msg_I = x_j (.) W   ->  MMA3_I: m_I^T += msg_I^T S_I^T  (S_I: pair -> i mod 128)
+//          msg_J = x_i (.) W   ->  MMA3_J: m_J^T += msg_J^T S_J^T  (m_I when I = J), from the
+//          same W once MMA3_I has read the message buffer
 //   DR     when a run of m_I or m_J ends (block row or block pair changes, or the CTA's run
 //          ends), the rows it touched are written as one fp32 partial block with a row mask;
 //          k_pair_sum adds them per row in a fixed order. No atomics, no edge-sized tensor.
 // Roles (22 warps, as in the directed kernel of tc_cfconv_ws.cu): prep 0-3, epilogue 4-19 (four
-// warps per TMEM lane quarter, 32 features each; per warp E2a(i), E1(i+1), E2b(i), DR(i)), MMA1
+// warps per TMEM lane quarter, 32 features each; per warp E2(i), E1(i+1), DR(i)), MMA1
 // warp 20, MMA2/MMA3 warp 21. TMEM: z1/u of two tiles (2 x 128 columns), m_I, m_J (128 each).
 // The 0/1 matrix S stays zero but for one entry per pair: each pair's thread clears the entry it
 // set for the previous product and sets the next one. Every wait is bounded.
@@ -388,37 +389,44 @@ __global__ void __launch_bounds__(PW_THREADS, 1) k_cfconv_pair_fwd(
       arrive_warp(B_FULL_H + b);
       return true;
     };
-    // a message y (.) W of tile i's filter, W = u + f_c c2, into H[b] as msg^T (MN-major)
-    auto message = [&](int i, const uint4* yv) {
+    // W = u + f_c c2 of tile i for this thread's 32 features (u read from TMEM)
+    auto filter = [&](int i, float* W) {
       const int b = i & 1;
       const float fc = MB(i % NMETA)->fc[e_me];
-      uint8_t* H = HB(b);
       uint32_t r[32];
       tc::ld32(lane_base + 128 * b + f0, r);
       tc::ld_wait();
 #pragma unroll
       for (int g8 = 0; g8 < 4; ++g8) {
+        const float4 ca = *(const float4*)(sc2 + f0 + 8 * g8);
+        const float4 cb = *(const float4*)(sc2 + f0 + 8 * g8 + 4);
+        const float cc[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+#pragma unroll
+        for (int k = 0; k < 8; ++k) W[8 * g8 + k] = fmaf(fc, cc[k], __uint_as_float(r[8 * g8 + k]));
+      }
+    };
+    // a message y (.) W into H[b] as msg^T (MN-major)
+    auto message = [&](int i, const uint4* yv, const float* W) {
+      uint8_t* H = HB(i & 1);
+#pragma unroll
+      for (int g8 = 0; g8 < 4; ++g8) {
         const uint4 yq = yv[g8];
         const uint32_t yw[4] = {yq.x, yq.y, yq.z, yq.w};
         const int f8 = f0 + 8 * g8;
-        const float4 ca = *(const float4*)(sc2 + f8);
-        const float4 cb = *(const float4*)(sc2 + f8 + 4);
-        const float cc[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
         uint32_t w[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int k = 8 * g8 + 2 * q;
-          const float W0 = fmaf(fc, cc[2 * q], __uint_as_float(r[k]));
-          const float W1 = fmaf(fc, cc[2 * q + 1], __uint_as_float(r[k + 1]));
-          w[q] = tc::pack_bf16(W0 * bf_lo(yw[q]), W1 * bf_hi(yw[q]));
-        }
+        for (int q = 0; q < 4; ++q)
+          w[q] = tc::pack_bf16(W[8 * g8 + 2 * q] * bf_lo(yw[q]),
+                               W[8 * g8 + 2 * q + 1] * bf_hi(yw[q]));
         *(uint4*)(H + (f8 >> 3) * 2048 + (e_me >> 3) * 128 + (e_me & 7) * 16) =
             make_uint4(w[0], w[1], w[2], w[3]);
       }
     };
-    // E2a of tile i: msg_I = x_j (.) W and S_I
-    auto E2a = [&](int i) -> bool {
+    // E2 of tile i: msg_I = x_j (.) W and S_I -> MMA3_I; once MMA3_I has read H[b] and S,
+    // msg_J = x_i (.) W (the same W, kept in registers) and S_J -> MMA3_J
+    auto E2 = [&](int i) -> bool {
       const int b = i & 1;
+      const PairMeta* M = MB(i % NMETA);
       if (!wait_warp(B_XFULL, i & 1)) return false;
       uint4 xv[FPT / 8];
 #pragma unroll
@@ -427,25 +435,37 @@ __global__ void __launch_bounds__(PW_THREADS, 1) k_cfconv_pair_fwd(
       if (lane == 0) mbar_arrive1(&bars[B_XFREE]);
       if (!wait_warp(B_DONE2 + b, (i >> 1) & 1)) return false;
       tc::fence_after();
-      message(i, xv);
+      float W[32];
+      filter(i, W);
+      message(i, xv, W);
+      // W kept for the second message as fp16 pairs (10-bit mantissa, below the message's bf16
+      // rounding), so that it holds 16 registers across the wait
+      uint32_t Wh[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const __half2 h = __floats2half2_rn(W[2 * k], W[2 * k + 1]);
+        Wh[k] = *(const uint32_t*)&h;
+      }
       if (part == 0) {  // MMA3_J of tile i-1 has completed (this warp saw it in DR(i-1))
         setS(rJ_prev, 0);
-        setS(MB(i % NMETA)->rI[e_me], 0x3F80);
+        setS(M->rI[e_me], 0x3F80);
       }
       arrive_warp(B_FULL_M + b);
-      return true;
-    };
-    // E2b of tile i: msg_J = x_i (.) W and S_J, once MMA3_I has read H[b] and S
-    auto E2b = [&](int i) -> bool {
-      const int b = i & 1;
-      const PairMeta* M = MB(i % NMETA);
-      const uint4* xr = (const uint4*)(x + (size_t)M->srcI[e_me] * FT + f0);
-      uint4 xv[FPT / 8];
+      uint4 xi[FPT / 8];  // x_i, requested while MMA3_I runs
+      {
+        const uint4* xr = (const uint4*)(x + (size_t)M->srcI[e_me] * FT + f0);
 #pragma unroll
-      for (int q = 0; q < FPT / 8; ++q) xv[q] = __ldg(xr + q);
+        for (int q = 0; q < FPT / 8; ++q) xi[q] = __ldg(xr + q);
+      }
       if (!wait_warp(B_DONE3A + b, (i >> 1) & 1)) return false;
       tc::fence_after();
-      message(i, xv);
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const float2 w2 = __half22float2(*(const __half2*)&Wh[k]);
+        W[2 * k] = w2.x;
+        W[2 * k + 1] = w2.y;
+      }
+      message(i, xi, W);
       if (part == 0) {
         setS(M->rI[e_me], 0);
         rJ_prev = M->rJ[e_me];
@@ -499,9 +519,8 @@ __global__ void __launch_bounds__(PW_THREADS, 1) k_cfconv_pair_fwd(
     bool ok = wait_warp(B_W, 0);  // c2 is read in the messages
     if (ok) ok = E1(0);
     for (int i = 0; ok && i < ntiles; ++i) {
-      ok = E2a(i);
+      ok = E2(i);
       if (ok && i + 1 < ntiles) ok = E1(i + 1);
-      if (ok) ok = E2b(i);
       if (ok) ok = DR(i);
     }
   }
