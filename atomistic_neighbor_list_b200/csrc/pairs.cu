@@ -27,7 +27,12 @@ namespace mp {
 namespace {
 
 constexpr int PB_THREADS = 512;
-constexpr int SUM_ROWS = 16;  // rows per k_pair_sum CTA
+constexpr int SUM_ROWS = 8;  // rows per k_pair_sum CTA (a multiple of 4)
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *(const uint32_t*)&h;
+}
 
 // Block-wide exclusive scan of one int per thread (blockDim.x a multiple of 32, at most 1024).
 __device__ int block_excl_scan(int v, int* s_warp, int* total) {
@@ -295,44 +300,55 @@ __global__ void k_pair_sumlist(int NB, const int* __restrict__ pbase_of,
   if (!FILL) sum_cnt[R] = n;
 }
 
-// out rows of block R, 16 per CTA (thread = feature): the sum of the partial blocks on R's list,
-// in list order, each row read only where the block's row mask has it; rows without pairs get 0.
+// out rows of block R, SUM_ROWS per CTA: the sum of the partial blocks on R's list, in list
+// order, each row read only where the block's row mask has it; rows without pairs get 0. Thread =
+// (row r0 + (t >> 5) + 4 m, features 4 (t & 31) .. + 3): 16-byte loads, many partials in flight.
 __global__ void __launch_bounds__(128) k_pair_sum(int N, const int* __restrict__ sum_ptr,
                                                   const int* __restrict__ sum_slots,
                                                   const float* __restrict__ part,
                                                   const uint32_t* __restrict__ pmask,
                                                   __nv_bfloat16* __restrict__ out) {
+  constexpr int RPT = SUM_ROWS / 4;  // rows per thread
   const int R = blockIdx.x / (128 / SUM_ROWS), rg = blockIdx.x % (128 / SUM_ROWS);
-  const int f = threadIdx.x, lr0 = rg * SUM_ROWS;
+  const int lr0 = rg * SUM_ROWS, fq = threadIdx.x & 31, rs = threadIdx.x >> 5;
   if (R * 128 + lr0 >= N) return;
-  float acc[SUM_ROWS];
+  float4 acc[RPT];
 #pragma unroll
-  for (int k = 0; k < SUM_ROWS; ++k) acc[k] = 0.f;
+  for (int m = 0; m < RPT; ++m) acc[m] = make_float4(0.f, 0.f, 0.f, 0.f);
   const int s0 = sum_ptr[R], s1 = sum_ptr[R + 1];
   __shared__ int s_slot[128];
   __shared__ uint32_t s_rows[128];
   for (int c0 = s0; c0 < s1; c0 += 128) {  // the list in chunks: slots and masks loaded at once
     const int m = min(128, s1 - c0);
-    if (f < m) {
-      const int slot = sum_slots[c0 + f];
-      s_slot[f] = slot;
-      s_rows[f] = __ldg(pmask + (size_t)slot * 4 + (lr0 >> 5)) >> (lr0 & 31);
+    if ((int)threadIdx.x < m) {
+      const int slot = sum_slots[c0 + threadIdx.x];
+      s_slot[threadIdx.x] = slot;
+      s_rows[threadIdx.x] = __ldg(pmask + (size_t)slot * 4 + (lr0 >> 5)) >> (lr0 & 31);
     }
     __syncthreads();
 #pragma unroll 4
     for (int q = 0; q < m; ++q) {
       const uint32_t rows = s_rows[q];
-      const float* p = part + ((size_t)s_slot[q] * 128 + lr0) * kPairF + f;
+      const float4* p = (const float4*)(part + ((size_t)s_slot[q] * 128 + lr0 + rs) * kPairF) + fq;
 #pragma unroll
-      for (int k = 0; k < SUM_ROWS; ++k)
-        if ((rows >> k) & 1u) acc[k] += __ldg(p + k * kPairF);
+      for (int k = 0; k < RPT; ++k) {
+        if ((rows >> (rs + 4 * k)) & 1u) {
+          const float4 v = __ldg(p + k * 4 * (kPairF / 4));
+          acc[k].x += v.x;
+          acc[k].y += v.y;
+          acc[k].z += v.z;
+          acc[k].w += v.w;
+        }
+      }
     }
     __syncthreads();
   }
 #pragma unroll
-  for (int k = 0; k < SUM_ROWS; ++k) {
-    const int r = R * 128 + lr0 + k;
-    if (r < N) out[(size_t)r * kPairF + f] = __float2bfloat16_rn(acc[k]);
+  for (int k = 0; k < RPT; ++k) {
+    const int r = R * 128 + lr0 + rs + 4 * k;
+    if (r < N)
+      *(uint2*)(out + (size_t)r * kPairF + 4 * fq) =
+          make_uint2(pack_bf16x2(acc[k].x, acc[k].y), pack_bf16x2(acc[k].z, acc[k].w));
   }
 }
 

@@ -44,7 +44,51 @@ def parse():
                     help="other workloads measured beside the main line (comma list; empty: none)")
     ap.add_argument("--profile-run", action="store_true",
                     help="short run for ncu: no clocks sampler, no e2e, no CPU baseline")
+    ap.add_argument("--profile-case", default="", choices=["", "attn16k", "pairs10k"],
+                    help="with --profile-run: a small case of one kernel instead of the step "
+                         "(attention forward at 16,384 atoms, K = 256; the undirected-pair cfconv "
+                         "at 10k atoms); --warmup calls, then --steps calls")
     return ap.parse_args()
+
+
+def profile_case(args):
+    """A small case of one kernel, for an ncu capture: args.warmup + args.steps calls."""
+    import dataclasses
+
+    import numpy as np
+    import torch
+
+    from atomistic_neighbor_list_b200 import mp, synth
+    torch.cuda.set_device(0)
+    n_calls = args.warmup + args.steps
+    if args.profile_case == "attn16k":
+        wl = dataclasses.replace(synth.WORKLOADS["cfg4"], n_atoms=16384)
+        pos, _ = synth.positions_for(wl)
+        p = torch.from_numpy(pos).cuda()
+        nbr, mask = mp.neighbor_padded(p, wl.r_c, wl.K)
+        ctx = mp.Context.from_workload(wl, synth.make_weights(wl), max_atoms=len(pos), max_edges=1)
+        x = torch.from_numpy(synth.node_features(len(pos), wl.F)).cuda().to(torch.bfloat16)
+        o = torch.empty_like(x)
+        for _ in range(n_calls):
+            ctx.attn_fwd(p, nbr, mask, x, o)
+    else:
+        wl = synth.WORKLOADS["cfg2"]
+        pos, _ = synth.positions_for(wl)
+        perm = mp.spatial_order(torch.from_numpy(pos).cuda(), wl.r_c).cpu().numpy()
+        p = torch.from_numpy(np.ascontiguousarray(pos[perm])).cuda()
+        rp, ci = mp.neighbor_csr(p, wl.r_c)
+        ctx = mp.Context.from_workload(wl, synth.make_weights(wl), max_atoms=len(pos),
+                                       max_edges=ci.numel())
+        x = torch.from_numpy(synth.node_features(len(pos), wl.F)).cuda().to(torch.bfloat16)
+        o = torch.empty_like(x)
+        ctx.pair_plan(rp, ci)
+        for _ in range(n_calls):
+            ctx.cfconv_fwd_pairs(0, p, x, o)
+    torch.cuda.synchronize()
+    ctx.status_sync()
+    ctx.close()
+    print(json.dumps({"profile_case": args.profile_case, "calls": n_calls}), flush=True)
+    return 0
 
 
 def rank_info():
@@ -507,6 +551,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         return reference_arm(args)
+    if args.profile_run and args.profile_case:
+        return profile_case(args)
     import numpy as np
     import torch
     import torch.distributed as dist
