@@ -371,11 +371,17 @@ int mp::energy_forces_launches(mp_ctx* c, int N, long long E, const float* pos, 
     // bf16 path: every atomwise layer and both cfconv passes on the tensor cores
     // consecutive atomwise layers that depend only on the row run as one launch (tc_dense2)
     auto img = [&](int kind, int b) { return c->tc_dense_img + tc_dense_off(kind, b, B); };
+    // the forward cfconv over undirected pairs when the context holds a plan of this very list
+    // (mp_pair_plan on these buffers; the caller builds it again whenever the list changes)
+    const PairPlan& P = c->pair;
+    const bool pairs = P.valid && P.N == N && P.E == E && P.list_row_ptr == row_ptr &&
+                       P.list_col_idx == col_idx && P.G == c->num_sms;
     MP_TRY(launch_embed(c, N, types, s));
     MP_TRY(tc_dense(c, N, F, F, c->x_res, false, img(0, 0), c->b_in[0], c->h[0], true,
                     TC_DENSE_STORE, s));
     for (int b = 0; b < B; ++b) {
-      MP_TRY(tc_cfconv_fwd(c, b, N, E, pos, row_ptr, col_idx, c->h[b], c->m, s));
+      MP_TRY(pairs ? tc_cfconv_fwd_pairs(c, b, N, pos, c->h[b], c->m, s)
+                   : tc_cfconv_fwd(c, b, N, E, pos, row_ptr, col_idx, c->h[b], c->m, s));
       if (b + 1 < B)  // x += m W_out + b_out, then h of the next block = x W_in + b_in
         MP_TRY(tc_dense2(c, N, F, c->m, true, img(1, b), c->b_out[b], c->x_res, TC_DENSE_RESIDUAL,
                          img(0, b + 1), c->b_in[b + 1], F, c->h[b + 1], TC_DENSE_STORE, s));

@@ -59,6 +59,8 @@ struct PairPlan {
   bool valid = false;
   int N = 0, NB = 0, G = 0, T = 0, nslots = 0;
   long long E = 0;
+  const int* list_row_ptr = nullptr;  // the list the plan was built from (mp_energy_forces uses
+  const int* list_col_idx = nullptr;  // the pair forward for calls on these same buffers)
   void* ws = nullptr;      // per-block arrays (sized by E and the number of blocks)
   size_t ws_bytes = 0;
   void* tws = nullptr;     // the tiles (sized by their count)

@@ -383,6 +383,10 @@ int pair_plan_build(mp_ctx* ctx, int N, long long E, const int* row_ptr, const i
   PairPlan& P = ctx->pair;
   P.valid = false;
   if (N < 0 || E < 0 || E > INT32_MAX) return MP_ERR_INVALID_ARG;
+  if (ctx->ef_graph) {  // a recorded energy/forces graph may hold the previous plan's buffers
+    cudaGraphExecDestroy(ctx->ef_graph);
+    ctx->ef_graph = nullptr;
+  }
   const int NB = (N + 127) / 128;
   if (NB > (1 << 16)) return MP_ERR_CAPACITY;  // the lower-block bitmap of k_pair_blocks
   // phase 1: per block, arrays indexed by the list's offsets (pairs, segments, lower blocks)
@@ -413,6 +417,8 @@ int pair_plan_build(mp_ctx* ctx, int N, long long E, const int* row_ptr, const i
   P.E = E;
   P.NB = NB;
   P.G = ctx->num_sms;
+  P.list_row_ptr = row_ptr;
+  P.list_col_idx = col_idx;
   // a block's upper pairs are sorted in shared memory: at most 32 Ki of them (128 KB; a power of
   // two, the bitonic sort's padded length)
   const int kcap = 32 * 1024;

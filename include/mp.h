@@ -182,6 +182,11 @@ int mp_cfconv_fwd(mp_ctx* ctx, int block, int N, long long E, const float* pos,
  * column index outside [0, N)), MP_ERR_CUDA, CSR errors (validate).                            */
 int mp_pair_plan(mp_ctx* ctx, int N, long long E, const int* row_ptr, const int* col_idx,
                  void* stream);
+/* mp_energy_forces (bf16 tensor-core configuration) runs its forward cfconv passes over the pairs
+ * of this plan when it is called with the same N, E, row_ptr and col_idx buffers the plan was
+ * built from: the plan stands for the list those buffers held at mp_pair_plan time, so a caller
+ * that rewrites the list in place must call mp_pair_plan again (or build the plan of another list)
+ * before the next mp_energy_forces. Calls on other buffers use the directed kernels.           */
 
 /* mp_cfconv_fwd over the pairs of the current plan: the filter W(d_ij) = W(d_ji) evaluated once
  * per pair and both messages taken from it, x_j (.) W to row i and x_i (.) W to row j, on the

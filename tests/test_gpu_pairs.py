@@ -153,3 +153,37 @@ def test_pair_cfconv_needs_the_tensor_core_configuration(mp):
     with pytest.raises(mp.MpError) as e:
         ctx.cfconv_fwd_pairs(0, dev(pos), dev(synth.node_features(100, wl.F)))
     assert e.value.name == "MP_ERR_UNIMPLEMENTED"
+
+
+def test_energy_forces_uses_the_plan_of_its_own_list(mp):
+    # with a plan of the very buffers it is given, energy + forces run the pair forward (the
+    # profile shows it) and agree with the oracle; on a copy of the list they run the directed
+    # kernels and repeat the plan-free result bit for bit
+    from helpers import TOL_BF16_FORCE, rel_rms
+    wl, pos, gp, rp, ci = system(mp, "cfg2", 3000)
+    n = len(pos)
+    w = synth.make_weights(wl)
+    types = synth.atom_types(n, wl.n_types)
+    ctx = mp.Context.from_workload(wl, w, max_atoms=n, max_edges=ci.numel())
+    pd, td = dev(pos), dev(types)
+    e0, f0 = ctx.energy_forces(pd, td, rp, ci)
+    e0, f0 = e0.clone(), f0.clone()
+    ctx.pair_plan(rp, ci)
+    ctx.profile_begin()
+    e1, f1 = ctx.energy_forces(pd, td, rp, ci)
+    prof = ctx.profile_end()
+    e1, f1 = e1.clone(), f1.clone()
+    assert "cfconv_pair_tc" in prof and "cfconv_fwd_tc" not in prof
+    rp2, ci2 = rp.clone(), ci.clone()
+    ctx.profile_begin()
+    e2, f2 = ctx.energy_forces(pd, td, rp2, ci2)
+    prof2 = ctx.profile_end()
+    torch.cuda.synchronize()
+    ctx.status_sync()
+    assert "cfconv_fwd_tc" in prof2 and "cfconv_pair_tc" not in prof2
+    assert torch.equal(e2, e0) and torch.equal(f2, f0)
+    orp, oci = oracle_csr(pos, wl.r_c, rp, ci)
+    model = oracle.Model.from_workload(wl, oracle_weights(w, wl.dtype))
+    Eref, Fref, e_atom = oracle.energy_forces(model, pos, types, orp, oci, return_atom_energy=True)
+    assert abs(float(e1[0]) - Eref[0]) <= 2e-2 * np.abs(e_atom).sum()
+    assert rel_rms(f1.cpu().numpy(), Fref) <= TOL_BF16_FORCE
