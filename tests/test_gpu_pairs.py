@@ -187,3 +187,23 @@ def test_energy_forces_uses_the_plan_of_its_own_list(mp):
     Eref, Fref, e_atom = oracle.energy_forces(model, pos, types, orp, oci, return_atom_energy=True)
     assert abs(float(e1[0]) - Eref[0]) <= 2e-2 * np.abs(e_atom).sum()
     assert rel_rms(f1.cpu().numpy(), Fref) <= TOL_BF16_FORCE
+
+
+def test_pair_plan_reports_a_block_with_too_many_pairs(mp):
+    # a complete graph on 800 atoms: rows 0-127 hold 94,144 upper pairs, more than one block's
+    # sort holds; the plan reports the capacity error, leaves no plan behind, and the context goes
+    # on (its status word clear)
+    n = 800
+    rows = [np.delete(np.arange(n), i) for i in range(n)]
+    rp = np.concatenate([[0], np.cumsum([len(r) for r in rows])]).astype(np.int32)
+    ci = np.concatenate(rows).astype(np.int32)
+    wl = dataclasses.replace(synth.WORKLOADS["cfg2"], dtype="bf16")
+    ctx = mp.Context.from_workload(wl, synth.make_weights(wl), max_atoms=n, max_edges=len(ci))
+    with pytest.raises(mp.MpError) as e:
+        ctx.pair_plan(dev(rp), dev(ci))
+    assert e.value.name == "MP_ERR_CAPACITY"
+    with pytest.raises(mp.MpError) as e:
+        ctx.cfconv_fwd_pairs(0, dev(synth.uniform_positions(n, seed=1)),
+                             dev(synth.node_features(n, wl.F)).to(torch.bfloat16))
+    assert e.value.name == "MP_ERR_INVALID_ARG"
+    ctx.status_sync()
