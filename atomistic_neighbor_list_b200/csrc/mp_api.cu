@@ -296,6 +296,32 @@ extern "C" int mp_set_wait_budget(mp_ctx* c, long long ns) {
   return MP_OK;
 }
 
+extern "C" int mp_shard_graphs(const int* graph_ptr, int n_graphs, int rank, int world, int* g0,
+                               int* g1) {
+  if (!graph_ptr || n_graphs < 1 || world < 1 || rank < 0 || rank >= world || !g0 || !g1)
+    return MP_ERR_INVALID_ARG;
+  for (int g = 0; g < n_graphs; ++g)
+    if (graph_ptr[g + 1] < graph_ptr[g]) return MP_ERR_INVALID_ARG;
+  const long long a_begin = graph_ptr[0], total = (long long)graph_ptr[n_graphs] - a_begin;
+  // boundary k: the graph start nearest to the atom target a_begin + total k / world (the later
+  // one on a tie); nondecreasing in k, since the starts are
+  auto bound = [&](int k) {
+    if (k <= 0) return 0;
+    if (k >= world) return n_graphs;
+    const long long target = a_begin + total * k / world;
+    int lo = 0, hi = n_graphs;  // first start at or after the target (graph_ptr[n_graphs] is)
+    while (lo < hi) {
+      const int mid = (lo + hi) / 2;
+      if ((long long)graph_ptr[mid] < target) lo = mid + 1; else hi = mid;
+    }
+    if (lo > 0 && target - graph_ptr[lo - 1] < (long long)graph_ptr[lo] - target) --lo;
+    return lo;
+  };
+  *g0 = bound(rank);
+  *g1 = bound(rank + 1);
+  return MP_OK;
+}
+
 // ---------------------------------------------------------------------------------------------
 extern "C" int mp_cfconv_fwd(mp_ctx* c, int block, int N, long long E, const float* pos,
                              const int* row_ptr, const int* col_idx, const void* x, void* out,

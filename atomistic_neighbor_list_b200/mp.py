@@ -67,6 +67,7 @@ def _load():
         "mp_launch_count": (i64, [vp]),
         "mp_set_wait_budget": (i32, [vp, i64]),
         "mp_pair_plan": (i32, [vp, i32, i64, vp, vp, vp]),
+        "mp_shard_graphs": (i32, [vp, i32, i32, i32, POINTER(i32), POINTER(i32)]),
         "mp_cfconv_fwd_pairs": (i32, [vp, i32, i32, vp, vp, vp, vp]),
         "mp_set_graphs": (i32, [vp, i32]),
         "mp_md_verlet": (i32, [vp, i32, i64, vp, vp, vp, vp, c_float, i32, vp, vp, vp, vp, i32,
@@ -94,7 +95,7 @@ EXPORTED = ("mp_init", "mp_destroy", "mp_strerror", "mp_status_sync", "mp_neighb
             "mp_profile_begin", "mp_profile_end", "mp_profile_get", "mp_launch_count",
             "mp_attn_fwd_noalloc", "mp_selftest_tc", "mp_set_graphs",
             "mp_md_verlet", "mp_md_run", "mp_attn_bwd", "mp_attn_eq_fwd", "mp_spatial_order",
-            "mp_set_wait_budget", "mp_pair_plan", "mp_cfconv_fwd_pairs")
+            "mp_set_wait_budget", "mp_pair_plan", "mp_cfconv_fwd_pairs", "mp_shard_graphs")
 NOALLOC_MAX_NF = 524288  # MP_NOALLOC_MAX_NF: largest N * F mp_attn_fwd_noalloc accepts
 
 
@@ -441,6 +442,17 @@ def selftest_tc():
     out = (c_int * 2)()
     _check(lib.mp_selftest_tc(out), "mp_selftest_tc")
     return int(out[0]), int(out[1])
+
+
+def shard_graphs(graph_ptr, rank: int, world: int):
+    """mp_shard_graphs: the graphs [g0, g1) and atoms [a0, a1) of rank `rank` of `world`, for a
+    host int32 graph_ptr (numpy or a CPU tensor)."""
+    import numpy as np
+    gp = np.ascontiguousarray(np.asarray(graph_ptr, dtype=np.int32))
+    g0, g1 = c_int(0), c_int(0)
+    _check(lib.mp_shard_graphs(gp.ctypes.data_as(c_void_p), len(gp) - 1, rank, world,
+                               ctypes.byref(g0), ctypes.byref(g1)), "mp_shard_graphs")
+    return g0.value, g1.value, int(gp[g0.value]), int(gp[g1.value])
 
 
 def neighbor_csr(pos, r_c: float, graph_ptr=None, capacity: int | None = None, stream=None):

@@ -44,6 +44,10 @@ def parse():
                     help="other workloads measured beside the main line (comma list; empty: none)")
     ap.add_argument("--profile-run", action="store_true",
                     help="short run for ncu: no clocks sampler, no e2e, no CPU baseline")
+    ap.add_argument("--shard-replicas", action="store_true",
+                    help="N > 1: split the workload's graphs over the ranks (mp_shard_graphs; "
+                         "strong scaling of one multi-replica system) instead of one system per "
+                         "rank (weak scaling)")
     ap.add_argument("--profile-case", default="", choices=["", "attn16k", "pairs10k"],
                     help="with --profile-run: a small case of one kernel instead of the step "
                          "(attention forward at 16,384 atoms, K = 256; the undirected-pair cfconv "
@@ -113,11 +117,18 @@ def job_value(world: int, steps: int, max_ms: float) -> float:
     return world * steps / (max_ms / 1000.0)
 
 
-def rank_system(wl, rank: int):
-    """The system rank `rank` simulates: the workload's generator seeded by the rank, so the
-    ranks run independent replicas of the same size (positions float32 [N,3], graph_ptr)."""
+def rank_system(wl, rank: int, world: int = 1, shard: bool = False):
+    """The system rank `rank` simulates (positions float32 [N,3], graph_ptr): by default the
+    workload's generator seeded by the rank, so the ranks run independent replicas of the same
+    size; with shard, the rank's contiguous share of the workload's graphs (mp_shard_graphs),
+    rebased, so the ranks together run the one system."""
     from atomistic_neighbor_list_b200 import synth
-    return synth.positions_for(wl, seed=rank)
+    if not shard or world == 1:
+        return synth.positions_for(wl, seed=rank)
+    from atomistic_neighbor_list_b200 import mp
+    pos, gp = synth.positions_for(wl, seed=0)
+    g0, g1, a0, a1 = mp.shard_graphs(gp, rank, world)
+    return pos[a0:a1].copy(), (gp[g0:g1 + 1] - a0).copy()
 
 
 def load_peaks():
@@ -577,7 +588,11 @@ def main():
                                 device_id=torch.device(devn))
     peaks = load_peaks()
     wl = synth.WORKLOADS[args.workload]
-    pos, gp = rank_system(wl, rank)
+    shard = args.shard_replicas and world > 1
+    if shard and len(synth.positions_for(wl)[1]) - 1 < world:
+        raise SystemExit("--shard-replicas needs at least one graph per rank")
+    pos, gp = rank_system(wl, rank, world, shard)
+    jw = 1 if shard else world  # systems the job steps per step: one shared, or one per rank
     N = len(pos)
     types = synth.atom_types(N, wl.n_types)
     weights = synth.make_weights(wl)
@@ -633,7 +648,7 @@ def main():
     launches = ctx.launch_count() - launches0
     total_ms = sum(a.elapsed_time(b) for a, b in evs)
     max_ms = max_over_ranks(total_ms, world, devn)
-    value = job_value(world, args.steps, max_ms)
+    value = job_value(jw, args.steps, max_ms)
 
     # ---- per-kernel breakdown: the same steps again with the library's per-launch events (the
     # events add gaps between launches, so this pass is not part of `value`)
@@ -888,7 +903,7 @@ def main():
         bi = sum(x.numel() * x.element_size() for x in (h_pos, h_types, h_rp, h_ci)) + \
             (h_gp.numel() * 4 if G > 1 else 0)
         bo = h_energy.numel() * 4 + h_forces.numel() * 4
-        e2e = {"value": job_value(world, args.steps, e2e_ms), "unit": UNIT,
+        e2e = {"value": job_value(jw, args.steps, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo)}
     configs, cprofs = {}, {}
     if not args.profile_run and rank == 0 and args.configs:
@@ -923,7 +938,8 @@ def main():
     if rank == 0:
         res = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
                "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
-               "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+               "higher_is_better": True, "scaling": "strong" if shard else "weak",
+               "vs_baseline": None,
                "dtype": wl.dtype, "data": "synthetic",
                "config": {"workload": wl.name, "atoms": N, "edges": E, "blocks": wl.n_blocks,
                           "F": wl.F, "n_rbf": wl.n_rbf, "r_c": wl.r_c, "graphs": G,
@@ -931,7 +947,9 @@ def main():
                           "atom_order": "cell order (mp_spatial_order; a relabelling, done "
                                         "before timing)",
                           "launch": "energy_forces recorded once as a CUDA graph, replayed per step",
-                          "parallelism": f"replicas x{world} (independent systems, no collective)"},
+                          "parallelism": (f"graphs of one system sharded over {world} ranks "
+                                          "(mp_shard_graphs, no collective)") if shard else
+                                         f"replicas x{world} (independent systems, no collective)"},
                "attention_edges_per_s": attn,
                "md_loop": md,
                "edges_per_s_per_block": {"value": edges_per_s, "unit": "edges/s",

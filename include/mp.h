@@ -160,6 +160,16 @@ int mp_neighbor_padded(int N, const float* pos, const int* graph_ptr, int n_grap
 int mp_spatial_order(int N, const float* pos, const int* graph_ptr, int n_graphs, float cell,
                      int* perm, void* stream);
 
+/* Replica sharding over `world` ranks [FS: replicas are independent systems, simulated in one
+ * batch through graph_ptr]: rank `rank` takes the contiguous graphs [*g0, *g1), boundary k placed
+ * at the graph start nearest to the atom target graph_ptr[0] + total k / world (the later start
+ * on a tie), so every graph goes to exactly one rank, in order, and each rank's atom count is
+ * within one largest graph of total / world. A rank simulates its graphs with no communication (its own neighbor list,
+ * energy_forces on its atoms); an empty range ([g, g)) is possible when world > n_graphs.
+ * graph_ptr: HOST int32 [n_graphs + 1], nondecreasing. No device work.
+ * Errors: MP_ERR_INVALID_ARG.                                                                    */
+int mp_shard_graphs(const int* graph_ptr, int n_graphs, int rank, int world, int* g0, int* g1);
+
 /* One continuous-filter convolution [FS s.2.1-2.3] with block `block`'s filter weights:
  *   out_i = sum_{j in row i} x_j (.) W(|r_i - r_j|),   rows with no edges give 0.
  * x, out: [N][F] of the context dtype (float or bf16), 16-byte aligned (rows are read and
