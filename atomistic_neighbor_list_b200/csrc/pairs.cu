@@ -18,8 +18,7 @@
 //   k_pair_flags   for the kernel's split of the tiles over G CTAs: which tile starts an
 //                  accumulator run, which ends one, and the partial slot each run writes
 //   k_pair_sumlist per block of rows, the partial slots it sums, in a fixed order
-#include <algorithm>
-#include <cstdio>
+#include <climits>
 
 #include "mp_internal.cuh"
 
