@@ -329,7 +329,7 @@ def cpu_legs(key: str, full_units: float, budget_s: float = 3.0):
 
     import oracle
     from atomistic_neighbor_list_b200 import synth
-    wl = synth.WORKLOADS["cfg2" if key == "cfg2_block" else key]
+    wl = synth.WORKLOADS[{"cfg2_block": "cfg2", "cfg5_block": "cfg5"}.get(key, key)]
     model = oracle.Model.from_workload(wl, synth.make_weights(wl))
 
     if key in ("cfg1", "cfg2_block"):
@@ -345,6 +345,16 @@ def cpu_legs(key: str, full_units: float, budget_s: float = 3.0):
             t = time.perf_counter()
             oracle.cfconv(model, 0, pos, rp, ci, x, rows=rows)
             return time.perf_counter() - t, int(rp[n] - rp[0]), f"{n} of {len(pos)} rows"
+        unit, scale_kind = "edges/s", "edges"
+    elif key == "cfg5_block":  # one block's cfconv on a same-density smaller system
+        def run(frac):
+            n = max(64, int(wl.n_atoms * frac))
+            pos, _ = synth.positions_for(synth.scaled(wl, n))
+            rp, ci = oracle.neighbor_csr(pos, wl.r_c)
+            x = synth.node_features(n, wl.F)
+            t = time.perf_counter()
+            oracle.cfconv(model, 0, pos, rp, ci, x)
+            return time.perf_counter() - t, len(ci), f"all rows of a {n}-atom same-density system"
         unit, scale_kind = "edges/s", "edges"
     elif key == "cfg4":
         pos, _ = synth.positions_for(wl)
@@ -934,6 +944,8 @@ def main():
         for key, res in configs.items():
             units = res.get("edges", res.get("valid_edges"))
             res["cpu_baseline"] = cpu_legs(key, units)
+            if key == "cfg5":  # its cfconv block too
+                res["cpu_baseline_block"] = cpu_legs("cfg5_block", units)
 
     if rank == 0:
         res = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
