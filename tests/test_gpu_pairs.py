@@ -207,3 +207,25 @@ def test_pair_plan_reports_a_block_with_too_many_pairs(mp):
                              dev(synth.node_features(n, wl.F)).to(torch.bfloat16))
     assert e.value.name == "MP_ERR_INVALID_ARG"
     ctx.status_sync()
+
+
+def test_pair_kernel_bounded_waits_report_a_timeout_and_recover(mp):
+    # with a zero wait budget every hand-off wait of the pair kernel gives up at once: the kernel
+    # drains what it issued and returns, the status word reports MP_ERR_TIMEOUT; with the default
+    # budget the same context's next call matches the oracle
+    wl, pos, gp, rp, ci = system(mp, "cfg2", 1200)
+    ctx, w, x_t, x_ref, _ = run_pairs(mp, wl, pos, rp, ci)
+    ctx.set_wait_budget(0)
+    ctx.cfconv_fwd_pairs(0, dev(pos), x_t.to(DEV))
+    torch.cuda.synchronize()
+    with pytest.raises(mp.MpError) as e:
+        ctx.status_sync()
+    assert e.value.name == "MP_ERR_TIMEOUT"
+    ctx.set_wait_budget(2_000_000_000)
+    out = ctx.cfconv_fwd_pairs(0, dev(pos), x_t.to(DEV))
+    torch.cuda.synchronize()
+    ctx.status_sync()
+    orp, oci = oracle_csr(pos, wl.r_c, rp, ci)
+    model = oracle.Model.from_workload(wl, oracle_weights(w, wl.dtype))
+    ref = oracle.cfconv_pairs(model, 0, pos, orp, oci, x_ref)
+    assert normwise(out.float().cpu().numpy(), ref) <= TOL_BF16_FEAT
