@@ -348,8 +348,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1) k_attn_tc(
 #pragma unroll
         for (int qq = 0; qq < 4; ++qq) {
           const int k = 8 * g8 + 2 * qq;
-          w[qq] = tc::pack_bf16(ssp_scaled(__uint_as_float(r[k]), fc, fc * LN2),
-                                ssp_scaled(__uint_as_float(r[k + 1]), fc, fc * LN2));
+          w[qq] = ssp_scaled_bf16x2(__uint_as_float(r[k]), __uint_as_float(r[k + 1]), fc, fc * LN2);
         }
         *(uint4*)(H + kmaj(e_me, f0 + 8 * g8, K2)) = make_uint4(w[0], w[1], w[2], w[3]);
       }

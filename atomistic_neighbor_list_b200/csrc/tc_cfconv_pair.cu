@@ -381,8 +381,7 @@ __global__ void __launch_bounds__(PW_THREADS, 1) k_cfconv_pair_fwd(
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int k = 8 * g8 + 2 * q;
-          w[q] = tc::pack_bf16(ssp_scaled(__uint_as_float(r[k]), fc, fcln2),
-                               ssp_scaled(__uint_as_float(r[k + 1]), fc, fcln2));
+          w[q] = ssp_scaled_bf16x2(__uint_as_float(r[k]), __uint_as_float(r[k + 1]), fc, fcln2);
         }
         *(uint4*)(H + kmaj(e_me, f0 + 8 * g8, K2)) = make_uint4(w[0], w[1], w[2], w[3]);
       }

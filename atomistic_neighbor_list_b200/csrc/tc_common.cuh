@@ -42,6 +42,16 @@ __device__ __forceinline__ float ssp_scaled(float z, float fc, float fcln2) {
   return fmaf(fcln2, l, fc * fmaxf(z, 0.f));
 }
 
+// The same for two values, e^-|z| of both from one fp16-pair exponential: t <= 1 in fp16 is good
+// to 2^-11 relative (its argument rounded to fp16 adds at most about 2.6e-4 to t), below the bf16
+// rounding of the result that feeds the next MMA; returned packed as bf16 (lo = z0).
+__device__ __forceinline__ uint32_t ssp_scaled_bf16x2(float z0, float z1, float fc, float fcln2) {
+  const uint32_t th = tc::ex2h2(tc::pack_f16(-fabsf(z0) * LOG2E, -fabsf(z1) * LOG2E));
+  const float2 t = __half22float2(*reinterpret_cast<const __half2*>(&th));
+  const float l0 = tc::lg2f(fmaf(t.x, 0.5f, 0.5f)), l1 = tc::lg2f(fmaf(t.y, 0.5f, 0.5f));
+  return tc::pack_bf16(fmaf(fcln2, l0, fc * fmaxf(z0, 0.f)), fmaf(fcln2, l1, fc * fmaxf(z1, 0.f)));
+}
+
 // Named barrier over n threads; the _or form also returns the OR of pred over them.
 __device__ __forceinline__ void bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
