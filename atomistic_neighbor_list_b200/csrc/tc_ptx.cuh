@@ -282,11 +282,6 @@ __device__ __forceinline__ uint32_t ex2h2(uint32_t x) {
   asm("ex2.approx.f16x2 %0, %1;" : "=r"(r) : "r"(x));
   return r;
 }
-__device__ __forceinline__ uint32_t tanhh2(uint32_t x) {
-  uint32_t r;
-  asm("tanh.approx.f16x2 %0, %1;" : "=r"(r) : "r"(x));
-  return r;
-}
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
