@@ -86,3 +86,42 @@ def test_peaks_come_from_the_measured_file():
         assert p["bf16_tflops_sustained"] <= p["bf16_tflops"]
     else:
         assert p["source"] == "fallback" and p["hbm_gbs"] == 6650.0
+
+
+def test_work_model_of_the_pair_kernel_counts_one_filter_per_pair():
+    wl = synth.WORKLOADS["cfg2"]
+    E, N = 465_074, 10_000
+    _, fwd, _ = bench.kernel_model("cfconv_fwd_tc", wl, E, N)
+    bound, pair, unit = bench.kernel_model("cfconv_pair_tc", wl, E, N)
+    assert (bound, unit) == ("tensor", "TFLOP/s") and pair == fwd / 2
+
+
+PEAKS = {"hbm_gbs": 6554.9, "bf16_tflops": 1647.4, "bf16_tflops_sustained": 1381.5,
+         "sm_max_mhz": 1965.0, "source": "measured"}
+
+
+def test_roofline_takes_the_dominant_kernel_against_the_burst_peak():
+    wl = synth.WORKLOADS["cfg2"]
+    E, N = 465_074, 10_000
+    prof = {"cfconv_bwd_tc": {"total_ms": 3.0, "launches": 12},   # 0.25 ms per launch
+            "cfconv_fwd_tc": {"total_ms": 1.2, "launches": 12},
+            "dense_tc": {"total_ms": 0.5, "launches": 28}}
+    clocks = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    r = bench.roofline_of(prof, wl, E, N, PEAKS, clocks, per_unit_ms=6.0)
+    assert r["kernel"] == "cfconv_bwd_tc" and r["avg_launch_ms"] == 0.25
+    work = 2 * 45_568 * E
+    assert r["work_per_launch"] == work
+    assert abs(r["achieved"] - work / 0.25e-3 / 1e12) < 1e-9
+    assert r["peak"] == 1647.4 and abs(r["frac"] - r["achieved"] / 1647.4) < 1e-12
+    assert r["share_of_step"] == 0.5
+
+
+def test_power_capped_clocks_select_the_sustained_peak_and_alu_peaks_follow_the_clock():
+    capped = {"sm_mhz": 1300.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    assert bench.peak_for("tensor", PEAKS, capped)[0] == 1381.5
+    capped_high = {"sm_mhz": 1950.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    assert bench.peak_for("tensor", PEAKS, capped_high)[0] == 1647.4
+    alu, _ = bench.peak_for("alu", PEAKS, None)
+    assert abs(alu - 148 * 128 * 2 * 1965e6 / 1e12) < 1e-9
+    assert bench.peak_for("hbm", PEAKS, None)[0] == 6554.9
+    assert bench.roofline_of({}, synth.WORKLOADS["cfg2"], 1, 1, PEAKS, None) is None
