@@ -229,3 +229,19 @@ def test_pair_kernel_bounded_waits_report_a_timeout_and_recover(mp):
     model = oracle.Model.from_workload(wl, oracle_weights(w, wl.dtype))
     ref = oracle.cfconv_pairs(model, 0, pos, orp, oci, x_ref)
     assert normwise(out.float().cpu().numpy(), ref) <= TOL_BF16_FEAT
+
+
+def test_pair_cfconv_high_degree(mp):
+    # r_c = 10 A at the workloads' density in a 25 A box: about 250 neighbors per atom, some 16 k
+    # upper pairs per 128-atom block, block pairs of many tiles each
+    wl = dataclasses.replace(synth.WORKLOADS["cfg2"], dtype="bf16", r_c=10.0, n_atoms=1500)
+    pos = synth.uniform_positions(1500, seed=4)
+    perm = mp.spatial_order(dev(pos), wl.r_c).cpu().numpy()
+    pos = np.ascontiguousarray(pos[perm])
+    rp, ci = mp.neighbor_csr(dev(pos), wl.r_c)
+    assert ci.numel() > 200 * 1500
+    ctx, w, x_t, x_ref, out = run_pairs(mp, wl, pos, rp, ci, block=2)
+    orp, oci = oracle_csr(pos, wl.r_c, rp, ci)
+    model = oracle.Model.from_workload(wl, oracle_weights(w, wl.dtype))
+    ref = oracle.cfconv_pairs(model, 2, pos, orp, oci, x_ref)
+    assert normwise(out.float().cpu().numpy(), ref) <= TOL_BF16_FEAT
