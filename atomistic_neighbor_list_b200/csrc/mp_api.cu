@@ -16,8 +16,8 @@ const char* kernel_name(int id) {
       "cfconv_bwd_simt", "attn_simt", "validate_csr", "cfconv_fwd_tc", "cfconv_bwd_tc",
       "attn_tc", "dense_tc", "md_integrate", "attn_bwd_dst", "attn_bwd_src",
       "attn_transpose", "attn_eq_simt", "attn_bwd_dst_tc",
-      "attn_bwd_src_tc", "attn_eq_tc", "md_cutoff_list", "cfconv_fwd_tc_lockstep",
-      "cfconv_bwd_tc_lockstep", "pair_plan", "cfconv_pair_tc", "pair_sum"};
+      "attn_bwd_src_tc", "attn_eq_tc", "md_cutoff_list", "pair_plan", "cfconv_pair_tc",
+      "pair_sum"};
   return (id >= 0 && id < K_NUM) ? names[id] : "?";
 }
 

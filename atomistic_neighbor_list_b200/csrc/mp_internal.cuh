@@ -35,8 +35,8 @@ enum KernelId : int {
   K_EMBED = 0, K_DENSE, K_READOUT_E, K_READOUT_BWD, K_GRAPH_SUM, K_CFCONV_FWD_SIMT,
   K_CFCONV_BWD_SIMT, K_ATTN_SIMT, K_VALIDATE, K_CFCONV_FWD_TC, K_CFCONV_BWD_TC, K_ATTN_TC,
   K_DENSE_TC, K_MD, K_ATTN_BWD, K_ATTN_BWD_SRC, K_ATTN_REV, K_ATTN_EQ,
-  K_ATTN_BWD_TC, K_ATTN_BWD_SRC_TC, K_ATTN_EQ_TC, K_MD_CUT, K_CFCONV_FWD_TC_LS,
-  K_CFCONV_BWD_TC_LS, K_PAIR_PLAN, K_CFCONV_PAIR_TC, K_PAIR_SUM, K_NUM
+  K_ATTN_BWD_TC, K_ATTN_BWD_SRC_TC, K_ATTN_EQ_TC, K_MD_CUT, K_PAIR_PLAN, K_CFCONV_PAIR_TC,
+  K_PAIR_SUM, K_NUM
 };
 const char* kernel_name(int id);
 

@@ -15,16 +15,6 @@ int tc_cfconv_fwd(mp_ctx* ctx, int block, int N, long long E, const float* pos, 
 int tc_cfconv_fwd_ws(mp_ctx* ctx, int block, int N, long long E, const float* pos,
                      const int* row_ptr, const int* col_idx, const void* x, void* out,
                      cudaStream_t s);
-// One tile at a time, all warps in lock step (tc_cfconv.cu); used where the pipelined kernel's
-// shared-memory plan does not fit (16-bit Gaussian operand wider than 64 columns).
-int tc_cfconv_fwd_sequential(mp_ctx* ctx, int block, int N, long long E, const float* pos,
-                             const int* row_ptr, const int* col_idx, const void* x, void* out,
-                             cudaStream_t s);
-// Lock-step backward (tc_cfconv_bwd.cu); used where the pipelined kernel's shared-memory plan
-// does not fit.
-int tc_cfconv_bwd_sequential(mp_ctx* ctx, int block, int N, long long E, const float* pos,
-                             const int* row_ptr, const int* col_idx, const void* h, const void* g,
-                             float* grad_h, float* forces, bool accumulate, cudaStream_t s);
 // Warp-specialised pipelined variant of tc_cfconv_bwd (tc_cfconv_bwd_ws.cu).
 int tc_cfconv_bwd_ws(mp_ctx* ctx, int block, int N, long long E, const float* pos,
                      const int* row_ptr, const int* col_idx, const void* h, const void* g,

@@ -546,7 +546,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1) k_attn_tc(
 bool tc_attn_supported(const mp_ctx* ctx, int K) {
   const mp_config& c = ctx->cfg;
   return tc_supported(ctx) && ctx->tc_attn_p && ctx->tc_qk && c.n_heads == AH && c.head_dim == AD &&
-         K % TM == 0 && at_fits(k1_of(c.n_rbf), 1);
+         K % TM == 0 && k1_of(c.n_rbf) <= 64 && at_fits(k1_of(c.n_rbf), 1);  // built for 32-64
 }
 
 template <int NC>

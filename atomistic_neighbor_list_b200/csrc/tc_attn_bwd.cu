@@ -698,7 +698,8 @@ __global__ void __launch_bounds__(BT, 1) k_attn_bwd_src_tc(
 bool tc_attn_bwd_supported(const mp_ctx* ctx, int K) {
   const mp_config& c = ctx->cfg;
   return tc_supported(ctx) && ctx->tc_attn_p && c.n_heads == BH && c.head_dim == BD &&
-         K % TM == 0 && K <= KMAX && bw_fits_attn(k1_of(c.n_rbf)) && sr_fits(k1_of(c.n_rbf));
+         K % TM == 0 && K <= KMAX && k1_of(c.n_rbf) <= 64 &&  // built for 32-64 operand columns
+         bw_fits_attn(k1_of(c.n_rbf)) && sr_fits(k1_of(c.n_rbf));
 }
 
 int tc_attn_bwd_dst(mp_ctx* ctx, int N, int K, const float* pos, const int* nbr,

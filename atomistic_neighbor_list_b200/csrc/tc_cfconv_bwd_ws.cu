@@ -921,10 +921,6 @@ int tc_cfconv_bwd_ws(mp_ctx* ctx, int block, int N, long long E, const float* po
                      const int* row_ptr, const int* col_idx, const void* h, const void* g,
                      float* grad_h, float* forces, bool accumulate, cudaStream_t s) {
   const int K1 = k1_of(ctx->cfg.n_rbf);
-  // a Gaussian operand wider than the shared-memory plan allows: the lock-step kernel
-  if (!bw_fits(K1))
-    return tc_cfconv_bwd_sequential(ctx, block, N, E, pos, row_ptr, col_idx, h, g, grad_h, forces,
-                                    accumulate, s);
   const ImgLayout IL = img_layout(K1);
   const uint8_t* img = (const uint8_t*)ctx->tc_weights + IL.bytes * block;
   long long tiles = (E + TM - 1) / TM;

@@ -543,9 +543,6 @@ int tc_cfconv_fwd_ws(mp_ctx* ctx, int block, int N, long long E, const float* po
   const int K1 = k1_of(ctx->cfg.n_rbf);
   const ImgLayout IL = img_layout(K1);
   const uint8_t* img = (const uint8_t*)ctx->tc_weights + IL.bytes * block;
-  // a Gaussian operand wider than the shared-memory plan allows: the lock-step kernel
-  if (!ws_fits(K1))
-    return tc_cfconv_fwd_sequential(ctx, block, N, E, pos, row_ptr, col_idx, x, out, s);
   long long tiles = (E + TM - 1) / TM;
   int grid = ctx->num_sms;
   if (tiles < grid) grid = (int)(tiles > 0 ? tiles : 1);

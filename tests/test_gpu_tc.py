@@ -196,8 +196,8 @@ def test_bounded_wait_timeout_is_reported_and_the_context_recovers(mp):
 
 
 def test_sixty_four_radial_functions_run_warp_specialised(mp):
-    """The chain workload's 64 radial functions (a 16-bit Gaussian operand of 80 columns) run on
-    the warp-specialised forward and backward kernels, not on the lock-step fallbacks."""
+    """The chain workload's 64 radial functions (a 16-bit Gaussian operand of 80 columns, the
+    widest the tensor-core kernels take) run on the warp-specialised forward and backward."""
     wl = synth.WORKLOADS["cfg3"]
     pos, gp = synth.chain_replicas(4, 200, seed=3)
     n = len(pos)
@@ -212,4 +212,20 @@ def test_sixty_four_radial_functions_run_warp_specialised(mp):
     prof = ctx.profile_end()
     ctx.status_sync()
     assert "cfconv_fwd_tc" in prof and "cfconv_bwd_tc" in prof, prof
-    assert not any(k.endswith("_lockstep") for k in prof), prof
+
+
+def test_few_radial_functions_run_on_the_cuda_cores(mp):
+    """Eight radial functions (a 16-column operand, below the tensor-core kernels' 32 to 80) take
+    the bf16 path on the CUDA-core kernels, and energy and forces match the oracle."""
+    pos = synth.uniform_positions(600, seed=6)
+    wl = dataclasses.replace(synth.WORKLOADS["cfg2"], n_atoms=600, n_rbf=8)
+    rp, ci = mp.neighbor_csr(torch.from_numpy(pos).cuda(), wl.r_c)
+    ctx = mp.Context.from_workload(wl, synth.make_weights(wl), max_atoms=600, max_edges=ci.numel())
+    ctx.profile_begin()
+    ctx.energy_forces(torch.from_numpy(pos).cuda(),
+                      torch.from_numpy(synth.atom_types(600, wl.n_types)).cuda(), rp, ci)
+    prof = ctx.profile_end()
+    ctx.status_sync()
+    assert "cfconv_fwd_simt" in prof and "cfconv_fwd_tc" not in prof, prof
+    e_err, f_err, tol = run_ef(mp, pos, n_rbf=8)
+    assert e_err <= TOL_BF16_FEAT and f_err <= tol
